@@ -1,0 +1,248 @@
+/*
+ * CPU oracle for the forward pass of a sparse, noisy, top-k, capacity-limited
+ * Mixture-of-Experts layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg load this file's library.  The CUDA path never
+ * calls it and shares no code with it.
+ *
+ * Plain loops and double accumulation, written from the method's definition:
+ *   - "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター",
+ *     STEP 2 (router logits s_raw = W_g x), STEP 4 (s = s_raw + eps),
+ *     STEP 5 (KeepTopK: -inf outside the top k), STEP 6 (softmax over the
+ *     masked scores), STEP 8-10 (W_up, ReLU, W_down), STEP 11-12 (gate
+ *     scaling and weighted sum).
+ *   - "nanoMoEの深層解剖", slide 11 (router in full precision, autocast off),
+ *     slides 12-13 (topk, -inf scatter, softmax), slide 14 and slides 15-23
+ *     (one_hot + cumsum slot rank with all first choices ranked before all
+ *     second choices, capacity drop), slides 24-29 and 38-40 (combine with
+ *     the pre-drop gate, dropped pairs contribute nothing).
+ *
+ * Readings where the pages leave a step open:
+ *   - noise: s = fl32(s_raw + fl32(sigma * eps)) with eps ~ N(0,1) supplied;
+ *   - top-k order: descending score, ties to the lower expert index;
+ *   - capacity: C = min(N, ceil(cf * N * k / E)), cf = +inf means C = N;
+ *   - no gate renormalisation after drops; a token with every choice
+ *     dropped gets y = 0.
+ *
+ * Inputs are read at their exact values: fp32 arrays as float, bf16 arrays as
+ * their bit patterns widened exactly to float.  Build with -ffp-contract=off
+ * so that the two fp32 roundings of the noise step stay separate.
+ */
+#pragma STDC FP_CONTRACT OFF
+
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+
+static double elem(const void *p, int dt, size_t i)
+{
+    if (dt == ORACLE_BF16) {
+        uint32_t u = (uint32_t)((const uint16_t *)p)[i] << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)p)[i];
+}
+
+/* STEP 2 / slide 11: s_raw[t][e] = W_g[e] . x[t], summed in double, rounded
+ * once to fp32; then the router bias (if any) is added in fp32. */
+void oracle_router_logits(const void *x, int dt, const float *W_g, const float *b_g,
+                          int64_t N, int d, int E, float *s_raw)
+{
+    for (int64_t t = 0; t < N; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i)
+                acc += elem(x, dt, (size_t)t * d + i) * (double)W_g[(size_t)e * d + i];
+            float s = (float)acc;
+            if (b_g)
+                s = s + b_g[e];
+            s_raw[(size_t)t * E + e] = s;
+        }
+    }
+}
+
+/* Order used for KeepTopK: higher score first, equal scores by lower index. */
+static const float *g_sort_scores;
+static int before(const void *a, const void *b)
+{
+    int ia = *(const int *)a, ib = *(const int *)b;
+    float sa = g_sort_scores[ia], sb = g_sort_scores[ib];
+    if (sa > sb) return -1;
+    if (sa < sb) return 1;
+    return (ia < ib) ? -1 : (ia > ib);
+}
+
+/* STEP 3-6 / slides 12-13, starting from the router logits:
+ *   s      = fl32(s_raw + fl32(sigma * eps))        (noise; skipped if eps is NULL)
+ *   TopK   = the k experts first in (s desc, index asc) order, in that order
+ *   gates  = exp(s_j - s_top) / sum_l exp(s_l - s_top) over the kept experts
+ *            (the -inf entries contribute exp(-inf) = 0), in double, stored fp32.
+ * s_noisy (nullable) receives s. */
+void oracle_route_from_logits(const float *s_raw, const float *noise, float sigma,
+                              int64_t N, int E, int k,
+                              int32_t *topk_idx, float *gates, float *s_noisy)
+{
+    float *s = (float *)malloc(sizeof(float) * (size_t)E);
+    int *idx = (int *)malloc(sizeof(int) * (size_t)E);
+    for (int64_t t = 0; t < N; ++t) {
+        for (int e = 0; e < E; ++e) {
+            float v = s_raw[(size_t)t * E + e];
+            if (noise) {
+                float scaled = sigma * noise[(size_t)t * E + e];
+                v = v + scaled;
+            }
+            s[e] = v;
+            idx[e] = e;
+            if (s_noisy)
+                s_noisy[(size_t)t * E + e] = v;
+        }
+        g_sort_scores = s;
+        qsort(idx, (size_t)E, sizeof(int), before);
+        double top = (double)s[idx[0]];
+        double denom = 0.0;
+        for (int j = 0; j < k; ++j)
+            denom += exp((double)s[idx[j]] - top);
+        for (int j = 0; j < k; ++j) {
+            topk_idx[(size_t)t * k + j] = idx[j];
+            gates[(size_t)t * k + j] = (float)(exp((double)s[idx[j]] - top) / denom);
+        }
+    }
+    free(s);
+    free(idx);
+}
+
+/* Expert capacity C = min(N, ceil(cf * N * k / E)); cf = +inf gives N.
+ * Returns -1 for invalid arguments (cf <= 0 or NaN, k or E out of range). */
+int64_t oracle_capacity(int64_t N, int E, int k, double cf)
+{
+    if (N < 0 || E < 1 || k < 1 || k > E || !(cf > 0.0))
+        return -1;
+    if (isinf(cf))
+        return N;
+    double c = ceil(cf * (double)N * (double)k / (double)E);
+    if (c > (double)N)
+        return N;
+    return (int64_t)c;
+}
+
+/* Slides 14-23: an assignment's place in its expert's queue is the number of
+ * earlier assignments to the same expert, where every token's j-th choice
+ * comes before every token's (j+1)-th choice and tokens keep their order
+ * within one choice rank.  Places >= C are dropped (slot -1).
+ * counts[e] is the number of kept assignments of expert e (used_capacity). */
+void oracle_assign_slots(const int32_t *topk_idx, int64_t N, int E, int k, int64_t C,
+                         int32_t *slot, int32_t *counts)
+{
+    int64_t *queue = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    for (int j = 0; j < k; ++j) {
+        for (int64_t t = 0; t < N; ++t) {
+            int e = topk_idx[(size_t)t * k + j];
+            int64_t place = queue[e]++;
+            slot[(size_t)t * k + j] = (place < C) ? (int32_t)place : -1;
+        }
+    }
+    for (int e = 0; e < E; ++e)
+        counts[e] = (int32_t)(queue[e] < C ? queue[e] : C);
+    free(queue);
+}
+
+/* STEP 8-10 for one token and one expert, in double:
+ *   z = W_up[e] x,  h = max(0, z),  o = W_down[e] h. */
+void oracle_expert_ffn(const void *x, int dt, const void *W_up, const void *W_down,
+                       int64_t t, int e, int d, int d_ff, double *h, double *o)
+{
+    for (int f = 0; f < d_ff; ++f) {
+        double z = 0.0;
+        size_t wrow = ((size_t)e * d_ff + f) * d;
+        for (int i = 0; i < d; ++i)
+            z += elem(W_up, dt, wrow + i) * elem(x, dt, (size_t)t * d + i);
+        h[f] = z > 0.0 ? z : 0.0;
+    }
+    for (int i = 0; i < d; ++i) {
+        double acc = 0.0;
+        size_t wrow = ((size_t)e * d + i) * d_ff;
+        for (int f = 0; f < d_ff; ++f)
+            acc += elem(W_down, dt, wrow + f) * h[f];
+        o[i] = acc;
+    }
+}
+
+struct combine_job {
+    const void *x, *W_up, *W_down;
+    int dt;
+    const int32_t *topk_idx, *slot;
+    const float *gates;
+    int d, d_ff, k;
+    const int64_t *tokens;
+    int64_t begin, end;
+    double *y;
+};
+
+/* STEP 11-12 / slides 38-40: y[t] = sum over kept choices j of
+ * gates[t][j] * E_{e_j}(x[t]); a dropped choice adds nothing and the kept
+ * gates are not renormalised. */
+static void *combine_range(void *arg)
+{
+    struct combine_job *jb = (struct combine_job *)arg;
+    double *h = (double *)malloc(sizeof(double) * (size_t)jb->d_ff);
+    double *o = (double *)malloc(sizeof(double) * (size_t)jb->d);
+    for (int64_t r = jb->begin; r < jb->end; ++r) {
+        int64_t t = jb->tokens[r];
+        double *yt = jb->y + (size_t)r * jb->d;
+        for (int i = 0; i < jb->d; ++i)
+            yt[i] = 0.0;
+        for (int j = 0; j < jb->k; ++j) {
+            if (jb->slot[(size_t)t * jb->k + j] < 0)
+                continue;
+            int e = jb->topk_idx[(size_t)t * jb->k + j];
+            double g = (double)jb->gates[(size_t)t * jb->k + j];
+            oracle_expert_ffn(jb->x, jb->dt, jb->W_up, jb->W_down, t, e, jb->d, jb->d_ff, h, o);
+            for (int i = 0; i < jb->d; ++i)
+                yt[i] += g * o[i];
+        }
+    }
+    free(h);
+    free(o);
+    return NULL;
+}
+
+/* Layer output for the listed tokens (y rows in list order, double).
+ * Work is split over tokens across nthreads plain threads; each token's
+ * arithmetic is the same as with one thread. */
+void oracle_ffn_combine(const void *x, int dt, const void *W_up, const void *W_down,
+                        const int32_t *topk_idx, const float *gates, const int32_t *slot,
+                        int d, int d_ff, int k, const int64_t *tokens, int64_t n_tokens,
+                        double *y, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > n_tokens)
+        nthreads = n_tokens > 0 ? (int)n_tokens : 1;
+    struct combine_job *jobs = (struct combine_job *)calloc((size_t)nthreads, sizeof *jobs);
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof *th);
+    for (int w = 0; w < nthreads; ++w) {
+        struct combine_job *jb = &jobs[w];
+        jb->x = x; jb->W_up = W_up; jb->W_down = W_down; jb->dt = dt;
+        jb->topk_idx = topk_idx; jb->slot = slot; jb->gates = gates;
+        jb->d = d; jb->d_ff = d_ff; jb->k = k; jb->tokens = tokens; jb->y = y;
+        jb->begin = n_tokens * w / nthreads;
+        jb->end = n_tokens * (w + 1) / nthreads;
+    }
+    if (nthreads == 1) {
+        combine_range(&jobs[0]);
+    } else {
+        for (int w = 0; w < nthreads; ++w)
+            pthread_create(&th[w], NULL, combine_range, &jobs[w]);
+        for (int w = 0; w < nthreads; ++w)
+            pthread_join(th[w], NULL);
+    }
+    free(jobs);
+    free(th);
+}

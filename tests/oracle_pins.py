@@ -1,0 +1,316 @@
+"""Checks that pin the CPU oracle to facts fixed outside it.
+
+Each check raises AssertionError on a mismatch.  They are plain functions so
+that the regular tests and the planted-mistake test (which swaps in a mutated
+build of the oracle) run the very same checks.
+
+Sources of truth used here, none of which is the oracle's own code:
+  * the nanoMoE slides' worked examples (tests/golden/*.txt, with citations),
+  * brute-force enumeration of expert subsets and of queue places,
+  * numpy/scipy float64 library routines (matmul, softmax),
+  * closed forms and invariants of the definition (gates sum to 1, sigma = 0
+    leaves the scores unchanged, k = E with no capacity limit is the dense
+    softmax mixture, E = 1 and k = 1 is a plain ReLU MLP).
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+from scipy.special import softmax as sp_softmax
+
+import oracle
+from tests.golden import load_m1, load_m2
+
+
+# ---------------------------------------------------------------- helpers
+def brute_topk(scores: np.ndarray, k: int):
+    """The k-subset S with min over S >= max outside S; among several (ties),
+    the one whose sorted index tuple is smallest.  Returned in (score desc,
+    index asc) order.  Only comparisons, no arithmetic."""
+    E = len(scores)
+    best = None
+    for S in itertools.combinations(range(E), k):
+        inside = [scores[i] for i in S]
+        outside = [scores[i] for i in range(E) if i not in S]
+        if outside and min(inside) < max(outside):
+            continue
+        if best is None or S < best:
+            best = S
+    return sorted(best, key=lambda i: (-scores[i], i))
+
+
+def brute_slots(topk: np.ndarray, E: int, C: int):
+    """Queue place of (t, j) = number of assignments to the same expert that
+    come earlier, where earlier means a lower choice rank j, or the same j and
+    a lower token index.  O((N k)^2)."""
+    N, k = topk.shape
+    slot = np.full((N, k), -1, dtype=np.int64)
+    for t in range(N):
+        for j in range(k):
+            e = topk[t, j]
+            place = 0
+            for t2 in range(N):
+                for j2 in range(k):
+                    if topk[t2, j2] == e and (j2 < j or (j2 == j and t2 < t)):
+                        place += 1
+            slot[t, j] = place if place < C else -1
+    counts = np.array([np.sum((topk == e) & (slot >= 0)) for e in range(E)])
+    return slot, counts
+
+
+def np_expert(x, W_up, W_down, e):
+    """numpy float64: W_down[e] @ max(0, W_up[e] @ x)."""
+    return W_down[e] @ np.maximum(W_up[e] @ x, 0.0)
+
+
+# ---------------------------------------------------------------- checks
+def check_m1():
+    """Slides 11-13: kept indices and 3-decimal gates of the 8 printed tokens."""
+    rows = load_m1()
+    logits = np.array([r[0] for r in rows], dtype=np.float32)
+    idx, g = oracle.route_from_logits(logits, 2)
+    for t, (lg, kept, gates) in enumerate(rows):
+        assert tuple(sorted(idx[t].tolist())) == kept, (t, idx[t], kept)
+        # descending order: the first choice has the larger logit
+        assert lg[idx[t][0]] >= lg[idx[t][1]]
+        by_index = {int(idx[t][j]): float(g[t][j]) for j in range(2)}
+        for e, expect in zip(kept, gates):
+            assert abs(by_index[e] - expect) <= 5e-4 + 1e-7, (t, e, by_index[e], expect)
+
+
+def check_m2_slots():
+    """Slides 15-23: queue places without a cut, and the cut at capacity 1."""
+    m2 = load_m2()
+    topk = np.array(m2["topk"], dtype=np.int32)
+    slot, counts = oracle.assign_slots(topk, m2["E"], C=topk.shape[0])
+    assert slot.tolist() == m2["rank_nocap"], slot.tolist()
+    slot, counts = oracle.assign_slots(topk, m2["E"], C=m2["C"])
+    assert slot.tolist() == m2["slot_cap1"], slot.tolist()
+    assert counts.tolist() == m2["used"], counts.tolist()
+
+
+def check_m2_combine(seed=3):
+    """Slides 24-29 and 38-40: token 0 gets 0.6 a + 0.3 a', token 1 gets 0.3 b,
+    tokens 2 and 3 get zero rows (their choices were all dropped)."""
+    m2 = load_m2()
+    rng = np.random.default_rng(seed)
+    N, E, k, d, d_ff = 4, m2["E"], m2["k"], 5, 7
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_up = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    topk = np.array(m2["topk"], dtype=np.int32)
+    gates = np.array(m2["gates"], dtype=np.float32)
+    slot = np.array(m2["slot_cap1"], dtype=np.int32)
+    y = oracle.ffn_combine(x, W_up, W_down, topk, gates, slot)
+    x64, u64, w64 = (a.astype(np.float64) for a in (x, W_up, W_down))
+    for t, terms in enumerate(m2["combine"]):
+        expect = np.zeros(d)
+        for g, e, tok in terms:
+            expect += np.float64(np.float32(g)) * np_expert(x64[tok], u64, w64, e)
+        np.testing.assert_allclose(y[t], expect, rtol=1e-12, atol=1e-12)
+
+
+def check_topk_bruteforce(seed=0, trials=300):
+    """KeepTopK (the walkthrough's STEP 5) against subset enumeration, with
+    random and deliberately tied scores; ties go to the lower index."""
+    rng = np.random.default_rng(seed)
+    for trial in range(trials):
+        E = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        if trial % 2:
+            s = rng.integers(-2, 3, size=E).astype(np.float32)  # many ties
+        else:
+            s = rng.standard_normal(E).astype(np.float32)
+        idx, g = oracle.route_from_logits(s[None, :], k)
+        assert idx[0].tolist() == brute_topk(s.tolist(), k), (s, k, idx[0])
+
+
+def check_gates_invariants(seed=1):
+    """STEP 6: kept gates sum to 1, masked experts get nothing (the kept set
+    has exactly k distinct experts), k = 1 gives gate 1 exactly, and gate
+    ratios follow exp(s_a - s_b)."""
+    rng = np.random.default_rng(seed)
+    for _ in range(50):
+        E = int(rng.integers(2, 17))
+        k = int(rng.integers(1, E + 1))
+        s = (3 * rng.standard_normal((6, E))).astype(np.float32)
+        idx, g = oracle.route_from_logits(s, k)
+        for t in range(6):
+            assert len(set(idx[t].tolist())) == k
+            assert abs(float(np.sum(g[t].astype(np.float64))) - 1.0) < 1e-6
+            assert np.all(g[t] > 0)
+            if k == 1:
+                assert g[t][0] == 1.0
+            for a in range(k):
+                for b in range(k):
+                    r = float(g[t][a]) / float(g[t][b])
+                    ref = math.exp(float(s[t, idx[t][a]]) - float(s[t, idx[t][b]]))
+                    assert abs(r - ref) <= 1e-5 * ref, (r, ref)
+
+
+def check_noise():
+    """STEP 3-4: sigma = 0 leaves the scores as they are; a noise draw can
+    reorder experts; the noisy score is the fp32 sum of s_raw and the fp32
+    product sigma * eps (two separate roundings)."""
+    rng = np.random.default_rng(7)
+    s_raw = rng.standard_normal((16, 6)).astype(np.float32)
+    eps = rng.standard_normal((16, 6)).astype(np.float32)
+    i0, g0, s0 = oracle.route_from_logits(s_raw, 2, eps, 0.0, return_scores=True)
+    i1, g1 = oracle.route_from_logits(s_raw, 2)
+    assert np.array_equal(s0.view(np.uint32), s_raw.view(np.uint32))
+    assert np.array_equal(i0, i1) and np.array_equal(g0.view(np.uint32), g1.view(np.uint32))
+    # reorder: s_raw favours expert 0, the noise favours expert 1
+    i2, _ = oracle.route_from_logits(np.array([[1.0, 0.0]], np.float32), 1,
+                                     np.array([[0.0, 2.0]], np.float32), 1.0)
+    assert i2[0, 0] == 1
+    i3, _ = oracle.route_from_logits(np.array([[1.0, 0.0]], np.float32), 1,
+                                     np.array([[0.0, 2.0]], np.float32), 0.25)
+    assert i3[0, 0] == 0
+    # two roundings: sigma = 1 + 2^-23, eps = 2^-24 - 2^-48.  The exact product
+    # is 2^-24 (1 + 2^-24 - 2^-47), which rounds to 2^-24; 1 + 2^-24 is then a
+    # tie and rounds to 1.  A fused multiply-add would round 1 + product up
+    # to 1 + 2^-23.
+    sr = np.array([[1.0, 0.0]], np.float32)
+    ep = np.array([[2.0 ** -24 - 2.0 ** -48, 0.0]], np.float32)
+    sig = np.float32(1.0 + 2.0 ** -23)
+    assert float(ep[0, 0]) == 2.0 ** -24 - 2.0 ** -48   # exactly representable
+    _, _, s4 = oracle.route_from_logits(sr, 1, ep, float(sig), return_scores=True)
+    assert s4[0, 0] == np.float32(1.0)
+    sigma = np.float32(0.75)
+    _, _, s5 = oracle.route_from_logits(s_raw, 2, eps, float(sigma), return_scores=True)
+    assert np.array_equal(s5, (s_raw + (sigma * eps).astype(np.float32)).astype(np.float32))
+
+
+def check_capacity():
+    """C = ceil(cf * N * k / E), at most N; cf = inf gives N."""
+    assert oracle.capacity(8192, 8, 2, 1.25) == 2560
+    assert oracle.capacity(16384, 8, 2, 1.25) == 5120
+    assert oracle.capacity(32768, 64, 6, 1.0) == 3072
+    assert oracle.capacity(64, 8, 2, math.inf) == 64
+    assert oracle.capacity(10, 3, 2, 1.0) == 7
+    assert oracle.capacity(4, 3, 2, 100.0) == 4
+    assert oracle.capacity(4, 3, 2, 0.0) == -1
+    assert oracle.capacity(4, 3, 2, float("nan")) == -1
+    assert oracle.capacity(4, 3, 4, 1.0) == -1
+
+
+def check_slots_bruteforce(seed=2, trials=60):
+    """Queue places and drops against the counting definition, plus the
+    invariants: per-expert load <= C, kept + dropped = N k, no drops when
+    C = N, and a later choice rank is never kept while an earlier one to the
+    same expert was dropped."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        N = int(rng.integers(1, 13))
+        E = int(rng.integers(1, 6))
+        k = int(rng.integers(1, E + 1))
+        topk = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+        C = int(rng.integers(0, N + 1))
+        slot, counts = oracle.assign_slots(topk, E, C)
+        bs, bc = brute_slots(topk, E, C)
+        assert np.array_equal(slot, bs) and np.array_equal(counts, bc)
+        assert np.all(counts <= C)
+        assert counts.sum() + np.sum(slot < 0) == N * k
+        for e in range(E):
+            kept_j = [j for t in range(N) for j in range(k) if topk[t, j] == e and slot[t, j] >= 0]
+            drop_j = [j for t in range(N) for j in range(k) if topk[t, j] == e and slot[t, j] < 0]
+            if kept_j and drop_j:
+                assert max(kept_j) <= min(drop_j)
+        slot_n, _ = oracle.assign_slots(topk, E, N)
+        assert np.all(slot_n >= 0)
+
+
+def check_logits_vs_numpy(seed=4):
+    """STEP 2: s_raw = W_g x, against numpy's float64 matmul rounded to fp32
+    (within one fp32 ulp, since numpy sums in another order), plus the fp32
+    bias; bf16 inputs are read at their exact values."""
+    from sparse_mixture_experts_noisy_b200.synth import f32_to_bf16_bits, bf16_bits_to_f32
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((9, 37)).astype(np.float32)
+    W_g = rng.standard_normal((5, 37)).astype(np.float32)
+    b_g = rng.standard_normal(5).astype(np.float32)
+    for xin, xval in ((x, x), (f32_to_bf16_bits(x), bf16_bits_to_f32(f32_to_bf16_bits(x)))):
+        ref = (xval.astype(np.float64) @ W_g.astype(np.float64).T).astype(np.float32)
+        got = oracle.router_logits(xin, W_g)
+        assert np.max(np.abs(got.view(np.int32) - ref.view(np.int32))) <= 1
+        got_b = oracle.router_logits(xin, W_g, b_g)
+        assert np.max(np.abs(got_b.view(np.int32) - (ref + b_g).view(np.int32))) <= 1
+    one = np.array([[0x3F80, 0xC000, 0x3E80]], dtype=np.uint16)  # 1.0, -2.0, 0.25
+    eye = np.eye(3, dtype=np.float32)
+    assert oracle.router_logits(one, eye).tolist() == [[1.0, -2.0, 0.25]]
+
+
+def check_ffn_vs_numpy(seed=5):
+    """STEP 8-10 against numpy float64 matmuls, fp32 and bf16 storage."""
+    from sparse_mixture_experts_noisy_b200.synth import f32_to_bf16_bits, bf16_bits_to_f32
+    rng = np.random.default_rng(seed)
+    E, d, d_ff = 3, 6, 11
+    x = rng.standard_normal((4, d)).astype(np.float32)
+    W_up = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    for conv in (lambda a: a, f32_to_bf16_bits):
+        xs, us, ws = conv(x), conv(W_up), conv(W_down)
+        val = (lambda a: a.astype(np.float64)) if xs.dtype == np.float32 else \
+              (lambda a: bf16_bits_to_f32(a).astype(np.float64))
+        for t in range(4):
+            for e in range(E):
+                h, o = oracle.expert_ffn(xs, us, ws, t, e)
+                np.testing.assert_allclose(h, np.maximum(val(us)[e] @ val(xs)[t], 0), rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(o, np_expert(val(xs)[t], val(us), val(ws), e), rtol=1e-12, atol=1e-12)
+
+
+def check_dense_mixture(seed=6):
+    """With k = E and no capacity limit, nothing is masked or dropped and the
+    layer is the dense softmax-gated mixture sum_e softmax(s)_e E_e(x)."""
+    rng = np.random.default_rng(seed)
+    N, d, E, d_ff = 7, 5, 4, 6
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_g = rng.standard_normal((E, d)).astype(np.float32)
+    W_up = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    out = oracle.forward(x, W_g, None, None, 0.0, E, math.inf, W_up, W_down)
+    p = sp_softmax(out["s_raw"].astype(np.float64), axis=1)
+    x64, u64, w64 = (a.astype(np.float64) for a in (x, W_up, W_down))
+    for t in range(N):
+        ref = sum(p[t, e] * np_expert(x64[t], u64, w64, e) for e in range(E))
+        np.testing.assert_allclose(out["y"][t], ref, rtol=1e-6, atol=1e-6)
+
+
+def check_single_expert_mlp(seed=8):
+    """E = 1, k = 1: gate 1, nothing dropped with cf = 1, y = W_down relu(W_up x)."""
+    rng = np.random.default_rng(seed)
+    N, d, d_ff = 5, 4, 9
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_g = rng.standard_normal((1, d)).astype(np.float32)
+    W_up = rng.standard_normal((1, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((1, d, d_ff)).astype(np.float32)
+    out = oracle.forward(x, W_g, None, None, 0.0, 1, 1.0, W_up, W_down)
+    assert np.all(out["gates"] == 1.0) and np.all(out["slot"][:, 0] == np.arange(N))
+    ref = np.maximum(x.astype(np.float64) @ W_up[0].T.astype(np.float64), 0) @ W_down[0].T.astype(np.float64)
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+
+
+def check_all_dropped_is_zero(seed=9):
+    """A token whose every choice overflowed gets a zero row, not a
+    renormalised one (slides 38-40, tokens 2 and 3)."""
+    rng = np.random.default_rng(seed)
+    N, d, E, d_ff, k = 6, 3, 2, 4, 1
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_g = np.zeros((E, d), np.float32)
+    b_g = np.array([1.0, 0.0], np.float32)      # every token picks expert 0
+    W_up = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    out = oracle.forward(x, W_g, b_g, None, 0.0, k, 1.0, W_up, W_down)   # C = 3
+    assert out["C"] == 3
+    assert out["slot"][:, 0].tolist() == [0, 1, 2, -1, -1, -1]
+    assert np.all(out["y"][3:] == 0.0)
+    ref0 = np_expert(x[0].astype(np.float64), W_up.astype(np.float64), W_down.astype(np.float64), 0)
+    np.testing.assert_allclose(out["y"][0], ref0, rtol=1e-12, atol=1e-12)
+
+
+ALL_CHECKS = [check_m1, check_m2_slots, check_m2_combine, check_topk_bruteforce,
+              check_gates_invariants, check_noise, check_capacity, check_slots_bruteforce,
+              check_logits_vs_numpy, check_ffn_vs_numpy, check_dense_mixture,
+              check_single_expert_mlp, check_all_dropped_is_zero]

@@ -1,0 +1,77 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins
+catch every one of them (CPU only).
+
+Each mutant is the oracle's C source with one textual change, compiled to a
+temporary library and swapped in for the duration of the pin checks."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle.oracle as O
+from tests import oracle_pins as P
+
+MUTANTS = {
+    "slots_token_major": (
+        "for (int j = 0; j < k; ++j) {\n        for (int64_t t = 0; t < N; ++t) {",
+        "for (int64_t t = 0; t < N; ++t) {\n        for (int j = 0; j < k; ++j) {"),
+    "noise_dropped": ("v = v + scaled;", "v = v + 0.0f * scaled;"),
+    "noise_fused": ("float scaled = sigma * noise[(size_t)t * E + e];\n                v = v + scaled;",
+                    "v = fmaf(sigma, noise[(size_t)t * E + e], v);"),
+    "ties_to_higher_index": ("return (ia < ib) ? -1 : (ia > ib);", "return (ia > ib) ? -1 : (ia < ib);"),
+    "ascending_scores": ("if (sa > sb) return -1;\n    if (sa < sb) return 1;",
+                         "if (sa < sb) return -1;\n    if (sa > sb) return 1;"),
+    "softmax_over_all_experts": ("for (int j = 0; j < k; ++j)\n            denom +=",
+                                 "for (int j = 0; j < E; ++j)\n            denom +="),
+    "relu_missing": ("h[f] = z > 0.0 ? z : 0.0;", "h[f] = z;"),
+    "w_up_transposed": ("z += elem(W_up, dt, wrow + i)",
+                        "z += elem(W_up, dt, (size_t)e * d_ff * d + (size_t)i * d_ff + f)"),
+    "w_down_transposed": ("acc += elem(W_down, dt, wrow + f)",
+                          "acc += elem(W_down, dt, (size_t)e * d * d_ff + (size_t)f * d + i)"),
+    "capacity_off_by_one": ("(place < C) ? (int32_t)place : -1", "(place <= C) ? (int32_t)place : -1"),
+    "dropped_pairs_contribute": ("if (jb->slot[(size_t)t * jb->k + j] < 0)\n                continue;", ""),
+    "capacity_floor": ("double c = ceil(", "double c = floor("),
+    "bf16_decode_shift": ("<< 16;", "<< 15;"),
+    "counts_include_drops": ("counts[e] = (int32_t)(queue[e] < C ? queue[e] : C);",
+                             "counts[e] = (int32_t)queue[e];"),
+    "bias_dropped": ("s = s + b_g[e];", "s = s + 0.0f * b_g[e];"),
+    "gate_not_applied": ("yt[i] += g * o[i];", "yt[i] += o[i];"),
+    "softmax_not_shifted_sign": ("denom += exp((double)s[idx[j]] - top);",
+                                 "denom += exp(top - (double)s[idx[j]]);"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(O._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-o", str(lib), str(path), "-lm", "-lpthread"])
+    return str(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    lib_path = _build_mutant(tmp_path, name, old, new)
+    O._load()
+    saved = O._lib
+    try:
+        mutant = ctypes.CDLL(lib_path)
+        for fn in ("oracle_router_logits", "oracle_route_from_logits", "oracle_capacity",
+                   "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine"):
+            getattr(mutant, fn).argtypes = getattr(saved, fn).argtypes
+            getattr(mutant, fn).restype = getattr(saved, fn).restype
+        O._lib = mutant
+        caught = []
+        for check in P.ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                caught.append(check.__name__)
+        assert caught, f"mutant {name} passed every pin"
+    finally:
+        O._lib = saved
