@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Throughput of the sparse noisy top-k MoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral|decode|nano|fine|toy]
+                    [--impl ours|reference]
+
+One step = one moe_forward call (router, dispatch, expert FFN, combine) over
+one batch of the workload's synthetic tokens, inputs resident in HBM.  Under
+torchrun every rank runs its own independent batch (data-parallel replicas,
+weak scaling, no collective on the data path); the time is the max over ranks.
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle instead
+(rank 0 only, bounded samples of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "MoE layer tokens/sec at 1 B200; % of bf16 tensor peak (prefill) / HBM BW (decode)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+KERNELS_PER_FORWARD = 7  # route, hist, scan, assign+gather, up GEMM, down GEMM, combine
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mixtral", choices=["mixtral", "decode", "nano", "fine", "toy"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the secondary decode measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ ranks
+class Dist:
+    def __init__(self, backend="nccl"):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float, device=None) -> float:
+        if not self.pg:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+
+
+def aggregate(tokens_per_rank: int, steps: int, world: int, max_seconds: float) -> dict:
+    """Whole-job throughput from the slowest rank's device time."""
+    total = tokens_per_rank * steps * world
+    return {"value": total / max_seconds, "ms_per_step": 1e3 * max_seconds / steps}
+
+
+# ------------------------------------------------------------------ clocks
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+            0x10: "sync_boost", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Reads SM clocks and clock-event reasons through NVML every 20 ms (read only)."""
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = getattr(props, "pci_bus_id", None)
+            if bus is not None:
+                busid = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(busid.encode())
+            else:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((sm, r))
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in _REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+def ffn_flops(R: int, d: int, d_ff: int) -> float:
+    """Expert GEMMs: up (R x d x d_ff) and down (R x d_ff x d), 2 flops per MAC."""
+    return 4.0 * R * d * d_ff
+
+
+def ffn_bytes(counts, d: int, d_ff: int, elem: int) -> float:
+    """Least HBM traffic of the expert FFN: every touched expert's W_up and
+    W_down once, the gathered rows read once, the hidden rows written and read
+    once, the expert outputs written once."""
+    R = int(sum(counts))
+    touched = sum(1 for c in counts if c > 0)
+    return elem * (touched * 2.0 * d * d_ff + R * d + 2.0 * R * d_ff + R * d)
+
+
+def ncu_traffic(kernel_tag: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel source (its hash matches); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "sparse_mixture_experts_noisy_b200", "csrc", "gemm_tc.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for line in open(path):
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == kernel_tag and parts[1] == h:
+                return float(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_sample_time(inp, wl, n_route: int, n_ffn: int, nthreads: int, rng):
+    """Times the oracle on a bounded sample and extrapolates to the whole batch.
+    Returns (seconds per batch, description)."""
+    import oracle
+    N = wl.N
+    n_route = max(1, min(n_route, N))
+    t0 = time.perf_counter()
+    lg = oracle.router_logits(inp.x[:n_route], inp.W_g, inp.b_g)
+    t_route = (time.perf_counter() - t0) * N / n_route
+    # routing + slot assignment on the full batch reuse the sampled logits
+    # pattern: tile the sample's logits to N rows (same arithmetic per row)
+    reps = int(math.ceil(N / n_route))
+    lg_full = np.tile(lg, (reps, 1))[:N]
+    noise = inp.noise
+    t0 = time.perf_counter()
+    idx, g = oracle.route_from_logits(lg_full, wl.k, noise, wl.sigma)
+    C = oracle.capacity(N, wl.E, wl.k, wl.cf)
+    slot, counts = oracle.assign_slots(idx, wl.E, C)
+    t_slots = time.perf_counter() - t0
+    toks = np.sort(rng.choice(N, size=max(1, min(n_ffn, N)), replace=False))
+    t0 = time.perf_counter()
+    oracle.ffn_combine(inp.x, inp.W_up, inp.W_down, idx, g, slot, tokens=toks, nthreads=nthreads)
+    t_ffn = (time.perf_counter() - t0) * N / len(toks)
+    desc = (f"router logits on {n_route} of {N} tokens, top-k/softmax/slots on all {N}, "
+            f"expert FFN + combine on {len(toks)} sampled tokens ({nthreads} threads); "
+            f"scaled to {N} tokens")
+    return t_route + t_slots + t_ffn, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def calibrated_ffn_tokens(wl, seconds: float, nthreads: int) -> int:
+    # about 1 ns per double multiply-add on one core for the oracle's plain loops
+    per_token = wl.k * 2.0 * wl.d * wl.d_ff * 1.0e-9
+    return max(1, min(wl.N, int(seconds * nthreads / max(per_token, 1e-9))))
+
+
+def run_reference(args):
+    from sparse_mixture_experts_noisy_b200.synth import WORKLOADS, make_inputs
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, args.seed)
+    cores = cpu_cores()
+    nthreads = max(1, min(cores, 64))
+    rng = np.random.default_rng(args.seed)
+    n_ffn = calibrated_ffn_tokens(wl, 2.0, nthreads)
+    n_route = min(wl.N, 2048)
+    for _ in range(args.warmup):
+        oracle_sample_time(inp, wl, min(n_route, 64), 1, nthreads, rng)
+    times = []
+    desc = ""
+    for _ in range(args.steps):
+        t, desc = oracle_sample_time(inp, wl, n_route, n_ffn, nthreads, rng)
+        times.append(t)
+    sec = float(np.mean(times))
+    value = wl.N / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, extra=None):
+    weights = 2 * wl.E * wl.d * wl.d_ff * (2 if wl.dtype == "bf16" else 4)
+    c = {"workload": wl.name, "N": wl.N, "d": wl.d, "E": wl.E, "d_ff": wl.d_ff, "k": wl.k,
+         "capacity_factor": wl.cf if math.isfinite(wl.cf) else "inf", "sigma": wl.sigma,
+         "router_bias_e0": wl.bias0, "storage": wl.dtype,
+         "l2": ("inputs larger than L2 (expert weights %.2f GB)" % (weights / 1e9)) if weights > L2_BYTES
+         else "L2 flushed between timed steps (256 MiB write)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ GPU arm
+def to_dev(a, torch):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def time_steps(fn, steps, torch, flush=None):
+    """Per-step CUDA events on the current stream; returns total seconds."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
+
+
+def measure_layer(wl, inp_dev, steps, warmup, dist, torch, moe, flush_needed):
+    x, W_g, b_g, noise, W_up, W_down = inp_dev
+    layer = moe.MoELayer(W_g, W_up, W_down, wl.k, wl.cf, b_g=b_g, sigma=wl.sigma, max_tokens=wl.N)
+    y = torch.empty_like(x)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=x.device) if flush_needed else None
+    flush = (lambda: flush_buf.fill_(1)) if flush_needed else None
+    run = lambda: layer(x, noise=noise, y=y)  # noqa: E731
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(x.device)
+    with clk:
+        sec = time_steps(run, steps, torch, flush)
+    torch.cuda.synchronize()
+    dist.barrier()
+    code, word = moe.check_status(layer.workspace)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} (0x{word:08x}) after the timed region")
+    return layer, y, sec, clk.summary()
+
+
+def measure_ffn(wl, inp_dev, steps, torch, moe):
+    """The dominant kernels alone: the expert FFN (tcgen05 grouped GEMMs) on the
+    batch's gathered rows, back to back on the current stream."""
+    x, W_g, b_g, noise, W_up, W_down = inp_dev
+    topk, gates, _ = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma, want_logits=False)
+    dsp = moe.moe_dispatch(topk, x, wl.E, wl.cf)
+    xg, offs, cnt = dsp["x_gathered"], dsp["offsets"], dsp["counts"]
+    rows, d = xg.shape
+    dt = moe.MOE_BF16 if xg.dtype == torch.bfloat16 else moe.MOE_F32
+    ws = torch.empty(moe.load_library().moe_expert_ffn_workspace_size(rows, d, wl.E, wl.d_ff, dt),
+                     dtype=torch.uint8, device=x.device)
+    out = torch.empty_like(xg)
+    run = lambda: moe.moe_expert_ffn(xg, offs, cnt, W_up, W_down, ws=ws, out=out)  # noqa: E731
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    sec = time_steps(run, steps, torch)
+    counts = cnt.cpu().numpy().tolist()
+    return sec / steps, counts
+
+
+def measure_e2e(layer, wl, inp, steps, torch, moe):
+    """Through the public API with host buffers: pinned x (and eps) copied in,
+    moe_forward, y copied out, every step."""
+    x_h = torch.from_numpy(inp.x.view(np.int16) if inp.x.dtype == np.uint16 else inp.x).pin_memory()
+    n_h = torch.from_numpy(inp.noise).pin_memory() if inp.noise is not None else None
+    x_d = torch.empty(x_h.shape, dtype=x_h.dtype, device="cuda")
+    n_d = torch.empty(n_h.shape, dtype=n_h.dtype, device="cuda") if n_h is not None else None
+    y_d = torch.empty(x_h.shape, dtype=x_h.dtype, device="cuda")
+    y_h = torch.empty(x_h.shape, dtype=x_h.dtype).pin_memory()
+    bf = inp.x.dtype == np.uint16
+
+    def step():
+        x_d.copy_(x_h, non_blocking=True)
+        if n_d is not None:
+            n_d.copy_(n_h, non_blocking=True)
+        xv = x_d.view(torch.bfloat16) if bf else x_d
+        layer(xv, noise=n_d, y=y_d.view(torch.bfloat16) if bf else y_d)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    sec = time_steps(step, steps, torch)
+    h2d = x_h.numel() * x_h.element_size() + (n_h.numel() * n_h.element_size() if n_h is not None else 0)
+    d2h = y_h.numel() * y_h.element_size()
+    return sec / steps, h2d, d2h
+
+
+def roofline_entry(kind, achieved, peak, unit, traffic, kernel, peak_src, extra=None):
+    e = {"bound": kind, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+         "traffic": traffic, "kernel": kernel, "peak_source": peak_src}
+    if extra:
+        e.update(extra)
+    return e
+
+
+def run_ours(args):
+    import torch
+    from sparse_mixture_experts_noisy_b200 import moe
+    from sparse_mixture_experts_noisy_b200.synth import WORKLOADS, make_inputs
+
+    dist = Dist("nccl")
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    moe.load_library()
+    peaks, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, args.seed + dist.rank)
+    inp_dev = tuple(to_dev(a, torch) for a in (inp.x, inp.W_g, inp.b_g, inp.noise, inp.W_up, inp.W_down))
+    weights_bytes = 2 * wl.E * wl.d * wl.d_ff * (2 if wl.dtype == "bf16" else 4)
+    flush = weights_bytes <= L2_BYTES
+
+    layer, y, sec, clocks = measure_layer(wl, inp_dev, args.steps, args.warmup, dist, torch, moe, flush)
+    max_sec = dist.max(sec, device=dev)
+    agg = aggregate(wl.N, args.steps, dist.world, max_sec)
+
+    # the dominant kernels alone
+    ffn_steps = max(10, min(args.steps, 200))
+    ffn_sec, counts = measure_ffn(wl, inp_dev, ffn_steps, torch, moe)
+    R = int(sum(counts))
+    elem = 2 if wl.dtype == "bf16" else 4
+    tc = wl.dtype == "bf16" and wl.d % 8 == 0 and wl.d_ff % 8 == 0
+    decode_plan = tc and moe.gathered_rows(wl.N, wl.E, wl.k, wl.cf) <= 256
+    kernel = "tc_gemm_kernel (up + down launches of one moe_expert_ffn call)" if tc else \
+             "simt_gemm_kernel (up + down)"
+    if decode_plan:
+        byt = ffn_bytes(counts, wl.d, wl.d_ff, elem)
+        roof = roofline_entry("hbm", byt / ffn_sec / 1e9, peaks["hbm_gbs"], "GB/s",
+                              ncu_traffic("decode"), kernel + " + reduce_parts_kernel", peak_src + " (copy)",
+                              {"algorithmic_bytes": byt, "ms_per_call": ffn_sec * 1e3})
+    else:
+        fl = ffn_flops(R, wl.d, wl.d_ff)
+        roof = roofline_entry("tensor", fl / ffn_sec / 1e12, peaks["bf16_tflops"], "TFLOP/s",
+                              ncu_traffic("prefill_" + wl.name), kernel, peak_src + " burst",
+                              {"frac_of_sustained": fl / ffn_sec / 1e12 / peaks["bf16_tflops_sustained"],
+                               "algorithmic_flops": fl, "kept_rows": R, "ms_per_call": ffn_sec * 1e3})
+        layer_tflops = fl / (max_sec / args.steps) / 1e12
+        roof["whole_layer_frac"] = layer_tflops / peaks["bf16_tflops"]
+
+    # end to end through the public API with host buffers
+    e2e_steps = max(5, min(args.steps, 50))
+    e2e_sec, h2d, d2h = measure_e2e(layer, wl, inp, e2e_steps, torch, moe)
+    e2e_sec = dist.max(e2e_sec, device=dev)
+
+    line = {"metric": METRIC, "value": agg["value"], "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, {"parallelism": f"replicas x{dist.world}" if dist.world > 1 else "1 GPU",
+                                           "seed": args.seed}),
+            "roofline": roof,
+            "e2e": {"value": wl.N * dist.world / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "clocks": clocks}
+
+    # the decode-shaped workload shares the weights' shapes and seeds with the
+    # Mixtral-shaped one; measure it too when running that workload
+    if args.workload == "mixtral" and not args.no_decode:
+        dwl = WORKLOADS["decode"]
+        dinp = make_inputs(dwl, args.seed + dist.rank, weights=False)
+        ddev = (to_dev(dinp.x, torch), inp_dev[1], None, None, inp_dev[4], inp_dev[5])
+        dsteps = max(20, args.steps)
+        dlayer, _, dsec, dclk = measure_layer(dwl, ddev, dsteps, args.warmup, dist, torch, moe, False)
+        dmax = dist.max(dsec, device=dev)
+        dagg = aggregate(dwl.N, dsteps, dist.world, dmax)
+        fsec, dcounts = measure_ffn(dwl, ddev, dsteps, torch, moe)
+        byt = ffn_bytes(dcounts, dwl.d, dwl.d_ff, 2)
+        layer_bytes = byt + dwl.N * dwl.d * 2 * 2 + dwl.E * dwl.d * 4
+        line["decode"] = {
+            "workload": "decode", "value": dagg["value"], "unit": UNIT, "ms_per_step": dagg["ms_per_step"],
+            "steps": dsteps,
+            "roofline": roofline_entry("hbm", byt / fsec / 1e9, peaks["hbm_gbs"], "GB/s", ncu_traffic("decode"),
+                                       "tc_gemm_kernel (decode tiles, up + down) + reduce_parts_kernel",
+                                       peak_src + " (copy)",
+                                       {"algorithmic_bytes": byt, "ms_per_call": fsec * 1e3,
+                                        "whole_layer_gbs": layer_bytes / (dmax / dsteps) / 1e9,
+                                        "whole_layer_frac": layer_bytes / (dmax / dsteps) / 1e9 / peaks["hbm_gbs"],
+                                        "whole_layer_frac_of_8tbs": layer_bytes / (dmax / dsteps) / 8e12}),
+            "clocks": dclk}
+        line["gpu_launches"] += KERNELS_PER_FORWARD * dsteps
+
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cores = cpu_cores()
+        nthreads = max(1, min(cores, 64))
+        rng = np.random.default_rng(args.seed)
+        n_ffn = calibrated_ffn_tokens(wl, args.cpu_seconds * 0.7, nthreads)
+        n_route = min(wl.N, max(256, int(args.cpu_seconds * 0.2 * 1e9 / max(1, wl.E * wl.d))))
+        t, desc = oracle_sample_time(inp, wl, n_route, n_ffn, nthreads, rng)
+        line["cpu_baseline"] = {"value": wl.N / t, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                                "sample": desc}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

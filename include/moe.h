@@ -1,0 +1,205 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) sparse noisy top-k Mixture-of-Experts
+ * layer forward pass (libmoe.so).
+ *
+ * The layer, as the MoE pages define it:
+ *   "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター" STEP 1-12 and
+ *   "nanoMoEの深層解剖" slides 11-40 (Router, MLPExperts, MOELayer):
+ *     s_raw = W_g x (+ b_g)                      router logits, fp32
+ *     s     = s_raw + sigma * eps                noise, eps supplied ~ N(0,1)
+ *     keep the k largest s, -inf elsewhere       KeepTopK
+ *     g     = softmax over the kept scores       gates
+ *     capacity-limited dispatch (first choices of all tokens ranked before
+ *       second choices, tokens in order; places >= C dropped)
+ *     E_e(x) = W_down[e] ReLU(W_up[e] x)         expert FFN
+ *     y     = sum over kept choices of g * E_e(x)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers marked "device" are device memory owned by the caller; the
+ *    library never allocates, frees or keeps them after the call returns.
+ *  - Scratch memory comes from a caller-provided workspace whose size the
+ *    matching *_workspace_size call returns (256-byte aligned start).
+ *  - Every compute call is asynchronous on the caller's CUDA stream
+ *    (cudaStream_t passed as void*; NULL is the legacy default stream).
+ *  - Arrays are dense and row-major.  Every array must start on a 16-byte
+ *    boundary.
+ *  - moe_dtype selects the storage type of x, W_up, W_down, the gathered
+ *    buffers and y.  W_g, b_g, noise, logits and gates are always fp32;
+ *    index arrays are int32.
+ *  - Return value: MOE_OK, or an error code with a message available from
+ *    moe_last_error() (thread-local, valid until the next call on that
+ *    thread).  Argument errors are detected on the host before anything is
+ *    launched.  Kernel-side failures (a bounded wait that ran out, an index
+ *    check) are recorded in the workspace's status word and returned by
+ *    moe_check_status().  No kernel traps.
+ *  - Preconditions: 1 <= k <= E <= 256; N >= 0; d, d_ff >= 1; inputs finite
+ *    (NaN or Inf in the scores gives unspecified routing).
+ *  - Ties in the top-k go to the lower expert index; the k kept experts of a
+ *    token are listed in (score descending, index ascending) order, which
+ *    defines the first, second, ... choice for capacity priority.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad size, null required pointer, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid arguments this build cannot run */
+    MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    MOE_ERR_DEVICE_CHECK = 5,  /* a kernel's own index check failed */
+    MOE_ERR_TIMEOUT = 6        /* a kernel's bounded wait ran out */
+} moe_status;
+
+/* Expert capacity C = min(N, ceil(cf * N * k / E)) computed in double
+ * ("nanoMoEの深層解剖" slide 14, get_capacity; the pages do not print its body,
+ * this is the problem statement's formula).  cf = +INFINITY means no limit
+ * (C = N).  Returns -1 if cf <= 0, cf is NaN, N < 0 or k, E are out of range. */
+MOE_API int64_t moe_capacity(int64_t N, int E, int k, double cf);
+
+/* Rows of the gathered (expert-major) buffers: min(N * k, E * C) rounded up
+ * to a multiple of 128.  x_gathered and out_gathered hold this many rows.
+ * Returns -1 on invalid arguments. */
+MOE_API int64_t moe_gathered_rows(int64_t N, int E, int k, double cf);
+
+/* ---------------------------------------------------------------- router */
+
+/* Router: logits, optional noise, KeepTopK and softmax over the kept scores.
+ * ("Mixture of Experts (MoE) 12段階…" STEP 2-6; "nanoMoEの深層解剖" slides 11-13.)
+ *
+ *  x          device [N, d] of dt
+ *  W_g        device [E, d] fp32            router weights, one row per expert
+ *  b_g        device [E] fp32 or NULL       router bias added in fp32 to W_g x
+ *  noise      device [N, E] fp32 or NULL    eps ~ N(0,1); skipped if NULL or sigma == 0
+ *  sigma      noise scale; s = fl32(s_raw + fl32(sigma * eps)) (two roundings, no FMA)
+ *  logits_out device [N, E] fp32 or NULL    receives s_raw (bias included, before noise)
+ *  topk_idx   device [N, k] int32           kept experts, first choice first
+ *  gates      device [N, k] fp32            softmax of the kept scores, same order
+ * The dot products accumulate in fp32 on CUDA cores (no tensor cores). */
+MOE_API moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                     const float *noise, float sigma, int64_t N, int d, int E, int k,
+                     float *logits_out, int32_t *topk_idx, float *gates, void *stream);
+
+/* ---------------------------------------------------------------- dispatch */
+
+/* Workspace bytes for moe_dispatch (per-block expert histograms). */
+MOE_API size_t moe_dispatch_workspace_size(int64_t N, int E, int k);
+
+/* Capacity-limited dispatch ("nanoMoEの深層解剖" slides 14-23, one_hot + cumsum
+ * ranking with all first choices before all second choices, capacity cut;
+ * slides 33-36 for the gathered expert batches).
+ *
+ *  topk_idx   device [N, k] int32 (from moe_route)
+ *  x          device [N, d] of dt
+ *  cf         capacity factor (see moe_capacity)
+ *  slot       device [N, k] int32 out: place of (t, j) in expert topk_idx[t][j]'s
+ *             queue, or -1 if dropped
+ *  counts     device [E] int32 out: kept rows per expert (<= C)
+ *  offsets    device [E + 1] int32 out: exclusive prefix sum of counts
+ *  x_gathered device [moe_gathered_rows(), d] of dt out: row offsets[e] + slot
+ *             holds x[t] for every kept (t, j) with topk_idx[t][j] = e.  Rows past
+ *             offsets[E] are left unwritten.
+ *  ws, ws_bytes  workspace, at least moe_dispatch_workspace_size() bytes
+ * Results are deterministic (no atomics decide an order). */
+MOE_API moe_status moe_dispatch(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N, int d,
+                        int E, int k, double cf, int32_t *slot, int32_t *counts,
+                        int32_t *offsets, void *x_gathered, void *ws, size_t ws_bytes,
+                        void *stream);
+
+/* ---------------------------------------------------------------- experts */
+
+/* Workspace bytes for moe_expert_ffn (status word + the hidden activations). */
+MOE_API size_t moe_expert_ffn_workspace_size(int64_t rows, int d, int E, int d_ff, moe_dtype dt);
+
+/* Expert FFN on the gathered rows ("Mixture of Experts (MoE) 12段階…" STEP 8-10;
+ * "nanoMoEの深層解剖" slide 32, MLPExperts with ReLU in place of GELU):
+ *   out[r] = W_down[e] ReLU(W_up[e] x_gathered[r])   for offsets[e] <= r < offsets[e] + counts[e]
+ *
+ *  x_gathered   device [rows, d] of dt
+ *  offsets      device [E + 1] int32, counts device [E] int32 (from moe_dispatch)
+ *  W_up         device [E, d_ff, d] of dt
+ *  W_down       device [E, d, d_ff] of dt
+ *  out_gathered device [rows, d] of dt; rows outside the kept ranges are unspecified
+ *  rows         allocated rows of x_gathered/out_gathered (moe_gathered_rows())
+ * bf16: tcgen05 tensor-core grouped GEMMs, fp32 accumulation, the hidden
+ * activation rounded to bf16 after ReLU, out rounded to bf16.  Needs d and
+ * d_ff multiples of 8; otherwise (and for fp32) CUDA-core fp32 kernels run.
+ * Rows are read from device counts, so nothing waits on the host. */
+MOE_API moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                          const void *W_up, const void *W_down, moe_dtype dt, int64_t rows,
+                          int d, int d_ff, int E, void *out_gathered, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* ---------------------------------------------------------------- combine */
+
+/* Gate-weighted combine back to token order ("Mixture of Experts (MoE) 12段階…"
+ * STEP 11-12; "nanoMoEの深層解剖" slides 38-40):
+ *   y[t] = sum over j with slot[t][j] >= 0 of gates[t][j] * out_gathered[offsets[e] + slot[t][j]]
+ * accumulated in fp32 in j order; a token with every choice dropped gets a
+ * zero row; gates are not renormalised after drops.
+ *  y device [N, d] of dt. */
+MOE_API moe_status moe_combine(const void *out_gathered, const int32_t *slot, const int32_t *topk_idx,
+                       const int32_t *offsets, const float *gates, moe_dtype dt, int64_t N,
+                       int d, int k, void *y, void *stream);
+
+/* ---------------------------------------------------------------- fused */
+
+/* Workspace bytes for moe_forward. */
+MOE_API size_t moe_workspace_size(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt);
+
+/* The whole layer: route, dispatch, expert FFN, combine, on one stream with no
+ * host synchronisation.  Arguments as in the calls above; every intermediate
+ * lives in ws.  logits_out/topk_out/gates_out/slot_out/counts_out (all nullable)
+ * receive copies of the intermediates for inspection.
+ *  y device [N, d] of dt. */
+MOE_API moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                       const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
+                       int k, double cf, const void *W_up, const void *W_down, void *y,
+                       float *logits_out, int32_t *topk_out, float *gates_out,
+                       int32_t *slot_out, int32_t *counts_out,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronises `stream` and reads the status word at the start of a workspace
+ * given to moe_expert_ffn or moe_forward.  Returns MOE_OK, MOE_ERR_TIMEOUT (a
+ * bounded wait in a kernel ran out; the kernel skipped its remaining work and
+ * released its tensor memory) or MOE_ERR_DEVICE_CHECK.  *detail (nullable)
+ * receives the raw word.  Clears the word. */
+MOE_API moe_status moe_check_status(void *ws, void *stream, uint32_t *detail);
+
+/* Diagnostic for the bounded-wait machinery: launches one CTA that waits on
+ * a shared-memory barrier nothing will ever complete, with a limit of
+ * timeout_us microseconds, using the same wait routine as the tensor-core
+ * kernels.  The kernel then records MOE_ERR_TIMEOUT in the status word of ws
+ * (>= 256 bytes) and returns.  No pages' counterpart; exists so that tests
+ * can check that a wait which runs out ends cleanly. */
+MOE_API moe_status moe_debug_wait_timeout(uint32_t timeout_us, void *ws, size_t ws_bytes, void *stream);
+
+/* Number of streaming multiprocessors the library sizes its persistent grids
+ * for on the current device (0 if no device). */
+MOE_API int moe_num_sms(void);
+
+MOE_API const char *moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

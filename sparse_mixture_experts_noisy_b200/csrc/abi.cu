@@ -1,0 +1,374 @@
+// The C ABI (include/moe.h): argument checks on the host, workspace carving,
+// and the launch sequence of the layer on one stream.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+moe_status fail(moe_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+moe_status cuda_fail(cudaError_t e, const char *where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
+
+int num_sms_current() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+bool use_tensor_cores(moe_dtype dt, int d, int d_ff) {
+    return dt == MOE_BF16 && d % 8 == 0 && d_ff % 8 == 0;
+}
+
+moe_status check_shape(int64_t N, int d, int E, int k, moe_dtype dt) {
+    if (dt != MOE_F32 && dt != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+    if (N < 0) return fail(MOE_ERR_INVALID_ARG, "N must be >= 0 (got %lld)", (long long)N);
+    if (d < 1) return fail(MOE_ERR_INVALID_ARG, "d must be >= 1 (got %d)", d);
+    if (E < 1 || E > 256) return fail(MOE_ERR_INVALID_ARG, "E must be in [1, 256] (got %d)", E);
+    if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, E] (got k=%d, E=%d)", k, E);
+    if (N * static_cast<int64_t>(k) > INT32_MAX)
+        return fail(MOE_ERR_INVALID_ARG, "N * k must fit in int32 (got %lld)", (long long)(N * k));
+    return MOE_OK;
+}
+
+#define REQUIRE_PTR(p, name)                                                                    \
+    do {                                                                                        \
+        if ((p) == nullptr) return fail(MOE_ERR_INVALID_ARG, "%s must not be NULL", name);      \
+        if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", name); \
+    } while (0)
+#define OPTIONAL_PTR(p, name)                                                                   \
+    do {                                                                                        \
+        if ((p) != nullptr && !aligned16(p))                                                    \
+            return fail(MOE_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);               \
+    } while (0)
+
+int64_t rows_for(int64_t N, int E, int k, int64_t C) {
+    int64_t r = N * k;
+    if (static_cast<int64_t>(E) * C < r) r = static_cast<int64_t>(E) * C;
+    return (r + 127) / 128 * 128;
+}
+
+size_t ffn_ws_bytes(int64_t rows, int d, int E, int d_ff, moe_dtype dt) {
+    if (use_tensor_cores(dt, d, d_ff)) return moe::tc_ffn_ws_bytes(rows, d, d_ff, E, num_sms_current());
+    return moe::align_up(static_cast<size_t>(rows) * d_ff * elem_bytes(dt), 256);
+}
+
+struct FwdLayout {
+    size_t status, topk, gates, slot, counts, offsets, dws, xg, og, ffn, total;
+};
+
+FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows, moe_dtype dt) {
+    using moe::align_up;
+    FwdLayout L{};
+    size_t o = 0;
+    L.status = o; o += moe::kStatusBytes;
+    const size_t nk = static_cast<size_t>(N) * k;
+    L.topk = o; o += align_up(nk * 4, 256);
+    L.gates = o; o += align_up(nk * 4, 256);
+    L.slot = o; o += align_up(nk * 4, 256);
+    L.counts = o; o += align_up(static_cast<size_t>(E) * 4, 256);
+    L.offsets = o; o += align_up(static_cast<size_t>(E + 1) * 4, 256);
+    L.dws = o; o += moe::dispatch_ws_bytes(N, E, k);
+    L.xg = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
+    L.og = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
+    L.ffn = o; o += ffn_ws_bytes(rows, d, E, d_ff, dt);
+    L.total = o;
+    return L;
+}
+
+moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts, const void *W_up,
+                   const void *W_down, moe_dtype dt, int64_t rows, int d, int d_ff, int E, void *out,
+                   void *ffn_ws, bool combine_reads_parts, float **parts_out, int *nparts_out,
+                   uint32_t *status, cudaStream_t s) {
+    cudaError_t e;
+    if (parts_out) *parts_out = nullptr;
+    if (nparts_out) *nparts_out = 0;
+    if (use_tensor_cores(dt, d, d_ff)) {
+        const int sms = num_sms_current();
+        const moe::TcPlan p = moe::plan_tc_ffn(rows, d, d_ff, E, sms);
+        uint8_t *w = static_cast<uint8_t *>(ffn_ws);
+        void *H = w;
+        float *parts = p.decode ? reinterpret_cast<float *>(w + moe::align_up(static_cast<size_t>(rows) * d_ff * 2, 256))
+                                : nullptr;
+        e = moe::launch_tc_ffn(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E, out, H, parts,
+                               combine_reads_parts, status, kWaitTimeoutNs, sms, s, nullptr);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core expert FFN launch");
+        if (p.decode && combine_reads_parts) {
+            if (parts_out) *parts_out = parts;
+            if (nparts_out) *nparts_out = p.splits_down;
+        }
+        return MOE_OK;
+    }
+    e = moe::launch_simt_ffn(xg, offsets, counts, W_up, W_down, dt == MOE_BF16 ? 1 : 0, rows, d, d_ff,
+                             E, out, ffn_ws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "CUDA-core expert FFN launch");
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+int moe_num_sms(void) { return num_sms_current(); }
+
+int64_t moe_capacity(int64_t N, int E, int k, double cf) {
+    if (N < 0 || E < 1 || E > 256 || k < 1 || k > E || !(cf > 0.0)) return -1;
+    if (std::isinf(cf)) return N;
+    const double c = std::ceil(cf * static_cast<double>(N) * static_cast<double>(k) / static_cast<double>(E));
+    if (c > static_cast<double>(N)) return N;
+    return static_cast<int64_t>(c);
+}
+
+int64_t moe_gathered_rows(int64_t N, int E, int k, double cf) {
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return -1;
+    return rows_for(N, E, k, C);
+}
+
+moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                     const float *noise, float sigma, int64_t N, int d, int E, int k,
+                     float *logits_out, int32_t *topk_idx, float *gates, void *stream) {
+    moe_status st = check_shape(N, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    if (N > 0) {
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(W_g, "W_g");
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(gates, "gates");
+        OPTIONAL_PTR(b_g, "b_g");
+        OPTIONAL_PTR(noise, "noise");
+        OPTIONAL_PTR(logits_out, "logits_out");
+    }
+    if (!std::isfinite(sigma)) return fail(MOE_ERR_INVALID_ARG, "sigma must be finite");
+    cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
+                                      logits_out, topk_idx, gates, nullptr,
+                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return MOE_OK;
+}
+
+size_t moe_dispatch_workspace_size(int64_t N, int E, int k) {
+    if (N < 0 || E < 1 || k < 1) return 0;
+    return moe::dispatch_ws_bytes(N, E, k);
+}
+
+moe_status moe_dispatch(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N, int d,
+                        int E, int k, double cf, int32_t *slot, int32_t *counts,
+                        int32_t *offsets, void *x_gathered, void *ws, size_t ws_bytes,
+                        void *stream) {
+    moe_status st = check_shape(N, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity factor must be > 0 or +inf (got %g)", cf);
+    REQUIRE_PTR(counts, "counts");
+    REQUIRE_PTR(offsets, "offsets");
+    if (N > 0) {
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(slot, "slot");
+        REQUIRE_PTR(x_gathered, "x_gathered");
+    }
+    const size_t need = moe::dispatch_ws_bytes(N, E, k);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "dispatch workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaError_t e = moe::launch_dispatch(topk_idx, x, elem_bytes(dt), N, d, E, k, C, slot, counts,
+                                         offsets, x_gathered, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    return MOE_OK;
+}
+
+size_t moe_expert_ffn_workspace_size(int64_t rows, int d, int E, int d_ff, moe_dtype dt) {
+    if (rows < 0 || d < 1 || E < 1 || d_ff < 1 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
+    return moe::kStatusBytes + ffn_ws_bytes(rows, d, E, d_ff, dt);
+}
+
+moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                          const void *W_up, const void *W_down, moe_dtype dt, int64_t rows,
+                          int d, int d_ff, int E, void *out_gathered, void *ws, size_t ws_bytes,
+                          void *stream) {
+    if (dt != MOE_F32 && dt != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+    if (rows < 0 || rows % 128 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "rows must be a non-negative multiple of 128 (moe_gathered_rows)");
+    if (d < 1 || d_ff < 1 || E < 1 || E > 256) return fail(MOE_ERR_INVALID_ARG, "bad d, d_ff or E");
+    if (rows > INT32_MAX) return fail(MOE_ERR_INVALID_ARG, "rows must fit in int32");
+    REQUIRE_PTR(offsets, "offsets");
+    REQUIRE_PTR(counts, "counts");
+    REQUIRE_PTR(W_up, "W_up");
+    REQUIRE_PTR(W_down, "W_down");
+    if (rows > 0) {
+        REQUIRE_PTR(x_gathered, "x_gathered");
+        REQUIRE_PTR(out_gathered, "out_gathered");
+    }
+    const size_t need = moe::kStatusBytes + ffn_ws_bytes(rows, d, E, d_ff, dt);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "expert FFN workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "status reset");
+    if (rows == 0) return MOE_OK;
+    return run_ffn(x_gathered, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, out_gathered,
+                   static_cast<uint8_t *>(ws) + moe::kStatusBytes, false, nullptr, nullptr, status, s);
+}
+
+moe_status moe_combine(const void *out_gathered, const int32_t *slot, const int32_t *topk_idx,
+                       const int32_t *offsets, const float *gates, moe_dtype dt, int64_t N,
+                       int d, int k, void *y, void *stream) {
+    if (dt != MOE_F32 && dt != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+    if (N < 0 || d < 1 || k < 1 || k > 256) return fail(MOE_ERR_INVALID_ARG, "bad N, d or k");
+    if (N > 0) {
+        REQUIRE_PTR(slot, "slot");
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(offsets, "offsets");
+        REQUIRE_PTR(gates, "gates");
+        REQUIRE_PTR(y, "y");
+        OPTIONAL_PTR(out_gathered, "out_gathered");
+    }
+    cudaError_t e = moe::launch_combine(out_gathered, nullptr, 0, 0, slot, topk_idx, offsets, gates,
+                                        dt == MOE_BF16 ? 1 : 0, N, d, k, 256, y,
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt) {
+    if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1) return 0;
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return 0;
+    return forward_layout(N, d, E, d_ff, k, rows_for(N, E, k, C), dt).total;
+}
+
+moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                       const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
+                       int k, double cf, const void *W_up, const void *W_down, void *y,
+                       float *logits_out, int32_t *topk_out, float *gates_out,
+                       int32_t *slot_out, int32_t *counts_out,
+                       void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = check_shape(N, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    if (d_ff < 1) return fail(MOE_ERR_INVALID_ARG, "d_ff must be >= 1");
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity factor must be > 0 or +inf (got %g)", cf);
+    if (!std::isfinite(sigma)) return fail(MOE_ERR_INVALID_ARG, "sigma must be finite");
+    REQUIRE_PTR(W_g, "W_g");
+    REQUIRE_PTR(W_up, "W_up");
+    REQUIRE_PTR(W_down, "W_down");
+    if (N > 0) {
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(y, "y");
+    }
+    OPTIONAL_PTR(b_g, "b_g");
+    OPTIONAL_PTR(noise, "noise");
+    OPTIONAL_PTR(logits_out, "logits_out");
+    OPTIONAL_PTR(topk_out, "topk_out");
+    OPTIONAL_PTR(gates_out, "gates_out");
+    OPTIONAL_PTR(slot_out, "slot_out");
+    OPTIONAL_PTR(counts_out, "counts_out");
+    const int64_t rows = rows_for(N, E, k, C);
+    if (rows > INT32_MAX) return fail(MOE_ERR_INVALID_ARG, "gathered rows must fit in int32");
+    const FwdLayout L = forward_layout(N, d, E, d_ff, k, rows, dt);
+    if (ws == nullptr || ws_bytes < L.total)
+        return fail(MOE_ERR_WORKSPACE, "forward workspace needs %zu bytes (got %zu)", L.total,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    uint32_t *status = reinterpret_cast<uint32_t *>(w + L.status);
+    int32_t *topk = topk_out ? topk_out : reinterpret_cast<int32_t *>(w + L.topk);
+    float *gates = gates_out ? gates_out : reinterpret_cast<float *>(w + L.gates);
+    int32_t *slot = slot_out ? slot_out : reinterpret_cast<int32_t *>(w + L.slot);
+    int32_t *counts = counts_out ? counts_out : reinterpret_cast<int32_t *>(w + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+    void *xg = w + L.xg;
+    void *og = w + L.og;
+
+    cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
+                                      logits_out, topk, gates, status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    if (N == 0) {
+        if (counts_out) {
+            e = cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * E, s);
+            if (e != cudaSuccess) return cuda_fail(e, "counts reset");
+        }
+        return MOE_OK;
+    }
+    e = moe::launch_dispatch(topk, x, elem_bytes(dt), N, d, E, k, C, slot, counts, offsets, xg,
+                             w + L.dws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    float *parts = nullptr;
+    int nparts = 0;
+    st = run_ffn(xg, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, og, w + L.ffn, true, &parts,
+                 &nparts, status, s);
+    if (st != MOE_OK) return st;
+    e = moe::launch_combine(og, parts, nparts, rows * static_cast<int64_t>(d), slot, topk, offsets,
+                            gates, dt == MOE_BF16 ? 1 : 0, N, d, k, E, y, s);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    return MOE_OK;
+}
+
+moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {
+    if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "ws must not be NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    e = cudaMemset(ws, 0, sizeof word);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    if (detail) *detail = word;
+    if (word & moe::ST_TIMEOUT)
+        return fail(MOE_ERR_TIMEOUT, "a kernel's bounded wait ran out (status 0x%08x)", word);
+    if (word & moe::ST_BOUNDS)
+        return fail(MOE_ERR_DEVICE_CHECK, "a kernel's index check failed (status 0x%08x)", word);
+    return MOE_OK;
+}
+
+moe_status moe_debug_wait_timeout(uint32_t timeout_us, void *ws, size_t ws_bytes, void *stream) {
+    if (ws == nullptr || ws_bytes < static_cast<size_t>(moe::kStatusBytes))
+        return fail(MOE_ERR_WORKSPACE, "needs a workspace of at least %d bytes", moe::kStatusBytes);
+    if (timeout_us == 0 || timeout_us > 2000000u)
+        return fail(MOE_ERR_INVALID_ARG, "timeout_us must be in [1, 2000000]");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess)
+        e = moe::launch_wait_timeout(static_cast<uint32_t *>(ws), static_cast<uint64_t>(timeout_us) * 1000ull, s);
+    if (e != cudaSuccess) return cuda_fail(e, "wait-timeout diagnostic launch");
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,161 @@
+// Gate-weighted combine back to token order.
+//
+// "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター" STEP 11 (g_i E_i(x)) and
+// STEP 12 (y = sum_i g_i E_i(x)); "nanoMoEの深層解剖" slides 38-40 (output =
+// cb_weight @ exp_out: a dropped pair has weight 0, the kept ones keep their
+// gate, so a token whose choices were all dropped gets a zero row).
+// The dense [tokens, E*C] x [E*C, d] product of the slides is replaced by a
+// gather: one warp per token reads its k expert-output rows and accumulates
+// g * row in fp32, in choice order j = 0..k-1.
+//
+// The expert outputs are either rows of dtype T (one partial) or `parts`
+// fp32 partial sums over K-splits of the down projection, which are added in
+// split order before the gate is applied.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCombineWarps = 8;
+
+template <typename T, int VEC>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16, 8> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
+        uint4 u = *reinterpret_cast<const uint4 *>(p);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(h[i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
+        uint4 u;
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(p) = u;
+    }
+};
+template <>
+struct Vec<float, 4> {
+    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
+        float4 u = *reinterpret_cast<const float4 *>(p);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+template <typename T>
+struct Vec<T, 1> {
+    static __device__ __forceinline__ void load(const T *p, float (&v)[1]) { v[0] = to_f32<T>(*p); }
+    static __device__ __forceinline__ void store(T *p, const float (&v)[1]) { *p = from_f32<T>(v[0]); }
+};
+
+template <int VEC>
+__device__ __forceinline__ void load_f32(const float *p, float (&v)[VEC]) {
+    if constexpr (VEC == 8) {
+        float4 a = *reinterpret_cast<const float4 *>(p);
+        float4 b = *reinterpret_cast<const float4 *>(p + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else if constexpr (VEC == 4) {
+        float4 a = *reinterpret_cast<const float4 *>(p);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else {
+        v[0] = *p;
+    }
+}
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kCombineWarps * 32)
+combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, int nparts,
+               int64_t part_stride, const int32_t *__restrict__ slot,
+               const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
+               const float *__restrict__ gates, int64_t N, int d, int k, int E,
+               T *__restrict__ y) {
+    extern __shared__ int32_t c_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t *rows = c_smem + warp * 2 * k;                       // [k] source row or -1
+    float *g = reinterpret_cast<float *>(rows + k);              // [k]
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
+    if (t >= N) return;
+    for (int j = lane; j < k; j += 32) {
+        const int32_t sl = slot[t * k + j];
+        const int32_t e = topk_idx[t * k + j];
+        const bool ok = sl >= 0 && e >= 0 && e < E;
+        rows[j] = ok ? offsets[e] + sl : -1;
+        g[j] = ok ? gates[t * k + j] : 0.0f;
+    }
+    __syncwarp();
+    for (int c = lane * VEC; c < d; c += 32 * VEC) {
+        float acc[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int32_t r = rows[j];
+            if (r < 0) continue;
+            float o[VEC];
+            if (nparts == 0) {
+                Vec<T, VEC>::load(out_rows + static_cast<int64_t>(r) * d + c, o);
+            } else {
+                load_f32<VEC>(parts + static_cast<int64_t>(r) * d + c, o);
+                for (int p = 1; p < nparts; ++p) {
+                    float q[VEC];
+                    load_f32<VEC>(parts + p * part_stride + static_cast<int64_t>(r) * d + c, q);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) o[v] += q[v];
+                }
+            }
+            const float gj = g[j];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj, o[v], acc[v]);
+        }
+        Vec<T, VEC>::store(y + t * d + c, acc);
+    }
+}
+
+template <typename T, int VEC>
+cudaError_t launch_combine_t(const void *out_rows, const float *parts, int nparts,
+                             int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
+                             const int32_t *offsets, const float *gates, int64_t N, int d, int k,
+                             int E, void *y, cudaStream_t s) {
+    const int64_t blocks = (N + kCombineWarps - 1) / kCombineWarps;
+    const size_t smem = sizeof(int32_t) * 2 * static_cast<size_t>(k) * kCombineWarps;
+    combine_kernel<T, VEC><<<static_cast<unsigned>(blocks), kCombineWarps * 32, smem, s>>>(
+        static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets,
+        gates, N, d, k, E, static_cast<T *>(y));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const void *out_rows, const float *parts, int nparts,
+                           int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
+                           const int32_t *offsets, const float *gates, int dt, int64_t N, int d,
+                           int k, int E, void *y, cudaStream_t s) {
+    if (N == 0) return cudaSuccess;
+    const bool al = (reinterpret_cast<uintptr_t>(y) % 16 == 0) &&
+                    (reinterpret_cast<uintptr_t>(out_rows) % 16 == 0) &&
+                    (reinterpret_cast<uintptr_t>(parts) % 16 == 0);
+    if (dt == 1) {
+        if (d % 8 == 0 && al)
+            return launch_combine_t<__nv_bfloat16, 8>(out_rows, parts, nparts, part_stride, slot,
+                                                      topk_idx, offsets, gates, N, d, k, E, y, s);
+        return launch_combine_t<__nv_bfloat16, 1>(out_rows, parts, nparts, part_stride, slot,
+                                                  topk_idx, offsets, gates, N, d, k, E, y, s);
+    }
+    if (d % 4 == 0 && al)
+        return launch_combine_t<float, 4>(out_rows, parts, nparts, part_stride, slot, topk_idx,
+                                          offsets, gates, N, d, k, E, y, s);
+    return launch_combine_t<float, 1>(out_rows, parts, nparts, part_stride, slot, topk_idx,
+                                      offsets, gates, N, d, k, E, y, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,203 @@
+// Capacity-limited dispatch: queue places, drops and the gathered expert batches.
+//
+// "nanoMoEの深層解剖" slides 14-23: exp_mask = one_hot(topk) permuted to
+// [k, tokens, E], cumsum over (k, tokens) - 1 gives each assignment its place in
+// its expert's queue (every first choice before every second choice, tokens in
+// order within a choice rank), places >= capacity are dropped, used_capacity
+// counts the kept ones.  Slides 33-36: the kept tokens are copied into one
+// buffer per expert.  The dense one-hot cumsum of the slides is replaced by
+// three passes whose result is the same number:
+//   1. hist:   per block of kDispatchTB tokens, per choice j, per expert e, the
+//              number of (t, j) in the block that chose e;
+//   2. scan:   for each (j, e), an exclusive prefix over blocks (in place) and
+//              the total over all tokens;
+//   3. assign: place(t, j) = sum_{j' < j} total[j'][e] + prefix over earlier
+//              blocks + rank among earlier tokens of the same block (warp
+//              match + per-warp counts), then slot = place < C ? place : -1, and
+//              the kept rows are copied to x_gathered[offsets[e] + place].
+// No step depends on the order in which threads or blocks run.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kDispatchTB = 256;               // tokens per block (one per thread)
+constexpr int kDispatchWarps = kDispatchTB / 32;
+
+__global__ void __launch_bounds__(kDispatchTB)
+hist_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k,
+            int32_t *__restrict__ hist /* [nblk][k][E] */) {
+    extern __shared__ int32_t h_smem[];  // [E]
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchTB + threadIdx.x;
+    for (int j = 0; j < k; ++j) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) h_smem[e] = 0;
+        __syncthreads();
+        if (t < N) {
+            const int e = topk_idx[t * k + j];
+            if (e >= 0 && e < E) atomicAdd(&h_smem[e], 1);
+        }
+        __syncthreads();
+        int32_t *dst = hist + (static_cast<int64_t>(blockIdx.x) * k + j) * E;
+        for (int e = threadIdx.x; e < E; e += blockDim.x) dst[e] = h_smem[e];
+        __syncthreads();
+    }
+}
+
+// One warp per (j, e): exclusive prefix of hist[b][j][e] over blocks b, in
+// place; the total goes to tot[j][e].
+__global__ void __launch_bounds__(256)
+scan_kernel(int32_t *__restrict__ hist, int nblk, int E, int k, int32_t *__restrict__ tot) {
+    const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (pair >= k * E) return;
+    const int64_t stride = static_cast<int64_t>(k) * E;
+    int32_t carry = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+        const int b = b0 + lane;
+        const int32_t v = (b < nblk) ? hist[b * stride + pair] : 0;
+        int32_t inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += u;
+        }
+        if (b < nblk) hist[b * stride + pair] = carry + inc - v;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) tot[pair] = carry;
+}
+
+__device__ __forceinline__ void copy_row(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                         int64_t bytes, bool vec16, int lane) {
+    if (vec16) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(src);
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+        for (int64_t i = lane; i < bytes / 16; i += 32) d[i] = s[i];
+    } else {
+        const uint16_t *s = reinterpret_cast<const uint16_t *>(src);
+        uint16_t *d = reinterpret_cast<uint16_t *>(dst);
+        for (int64_t i = lane; i < bytes / 2; i += 32) d[i] = s[i];
+    }
+}
+
+__global__ void __launch_bounds__(kDispatchTB)
+assign_kernel(const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ x, int64_t row_bytes,
+              bool vec16, int64_t N, int E, int k, int64_t C,
+              const int32_t *__restrict__ hist_excl /* [nblk][k][E] */,
+              const int32_t *__restrict__ tot /* [k][E] */, int32_t *__restrict__ slot,
+              int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+              uint8_t *__restrict__ x_gathered) {
+    extern __shared__ int32_t a_smem[];
+    int32_t *warp_cnt = a_smem;                                // [warps][E]
+    int32_t *jrun = warp_cnt + kDispatchWarps * E;             // [E]  sum_{j' < j} tot[j'][e]
+    int32_t *offs = jrun + E;                                  // [E + 1]
+    int32_t *rowmap = offs + E + 1;                            // [TB] destination row or -1
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchTB + tid;
+
+    // kept rows per expert and their exclusive prefix (every block computes the
+    // same values from tot; block 0 publishes them)
+    for (int e = tid; e < E; e += blockDim.x) {
+        int64_t total = 0;
+        for (int j = 0; j < k; ++j) total += tot[j * E + e];
+        offs[e] = static_cast<int32_t>(total < C ? total : C);
+        jrun[e] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int32_t run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t c = offs[e];
+            offs[e] = run;
+            run += c;
+            if (blockIdx.x == 0) counts[e] = c;
+        }
+        offs[E] = run;
+        if (blockIdx.x == 0)
+            for (int e = 0; e <= E; ++e) offsets[e] = offs[e];
+    }
+    __syncthreads();
+
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+        for (int i = tid; i < kDispatchWarps * E; i += blockDim.x) warp_cnt[i] = 0;
+        __syncthreads();
+        int e = -1;
+        if (t < N) {
+            e = topk_idx[t * k + j];
+            if (e < 0 || e >= E) e = -1;   // an out-of-range expert id is dropped
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank_in_warp = __popc(same & lt_mask);
+        if (e >= 0 && rank_in_warp == 0) warp_cnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        int32_t r = -1;
+        if (e >= 0) {
+            int64_t place = static_cast<int64_t>(jrun[e]) +
+                            hist_excl[(static_cast<int64_t>(blockIdx.x) * k + j) * E + e] + rank_in_warp;
+            for (int w = 0; w < warp; ++w) place += warp_cnt[w * E + e];
+            const bool kept = place < C;
+            slot[t * k + j] = kept ? static_cast<int32_t>(place) : -1;
+            if (kept) r = offs[e] + static_cast<int32_t>(place);
+        } else if (t < N) {
+            slot[t * k + j] = -1;
+        }
+        rowmap[tid] = r;
+        __syncthreads();
+        // copy the kept rows of this choice rank, one warp per row
+        for (int i = warp; i < kDispatchTB; i += kDispatchWarps) {
+            const int32_t dst = rowmap[i];
+            if (dst >= 0) {
+                const int64_t ts = static_cast<int64_t>(blockIdx.x) * kDispatchTB + i;
+                copy_row(x + ts * row_bytes, x_gathered + static_cast<int64_t>(dst) * row_bytes,
+                         row_bytes, vec16, lane);
+            }
+        }
+        for (int ee = tid; ee < E; ee += blockDim.x) jrun[ee] += tot[j * E + ee];
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+int64_t dispatch_blocks(int64_t N) { return (N + kDispatchTB - 1) / kDispatchTB; }
+
+size_t dispatch_ws_bytes(int64_t N, int E, int k) {
+    const int64_t nblk = dispatch_blocks(N);
+    const size_t hist = sizeof(int32_t) * static_cast<size_t>(nblk > 0 ? nblk : 1) * k * E;
+    const size_t tot = sizeof(int32_t) * static_cast<size_t>(k) * E;
+    return align_up(hist, 256) + align_up(tot, 256);
+}
+
+cudaError_t launch_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N,
+                            int d, int E, int k, int64_t C, int32_t *slot, int32_t *counts,
+                            int32_t *offsets, void *x_gathered, void *ws, cudaStream_t s) {
+    const int64_t nblk = dispatch_blocks(N);
+    int32_t *hist = static_cast<int32_t *>(ws);
+    int32_t *tot = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) +
+                                               align_up(sizeof(int32_t) * static_cast<size_t>(nblk > 0 ? nblk : 1) * k * E, 256));
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+        return e;
+    }
+    hist_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, sizeof(int32_t) * E, s>>>(topk_idx, N, E,
+                                                                                     k, hist);
+    const int pairs = k * E;
+    const int warps_per_block = 8;
+    scan_kernel<<<(pairs + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, s>>>(
+        hist, static_cast<int>(nblk), E, k, tot);
+    const int64_t row_bytes = static_cast<int64_t>(d) * elem_bytes;
+    const bool vec16 = (row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(x_gathered) % 16 == 0);
+    const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kDispatchWarps) * E + E + E + 1 + kDispatchTB);
+    assign_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, smem, s>>>(
+        topk_idx, static_cast<const uint8_t *>(x), row_bytes, vec16, N, E, k, C, hist, tot, slot,
+        counts, offsets, static_cast<uint8_t *>(x_gathered));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

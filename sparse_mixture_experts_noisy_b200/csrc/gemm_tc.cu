@@ -1,0 +1,523 @@
+// Expert FFN on the fifth-generation tensor cores: a persistent grouped GEMM
+// with tcgen05.mma (bf16 inputs, fp32 accumulators in tensor memory) fed by
+// TMA, one CTA per SM.
+//
+// "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター" STEP 8 (z = W_up x),
+// STEP 9 (ReLU, fused into the up-projection epilogue), STEP 10 (W_down h);
+// "nanoMoEの深層解剖" slide 32 (MLPExperts: one batched matmul per projection
+// over all experts).  The slides' bmm over a dense [E, capacity, d] batch is
+// replaced by a grouped GEMM over the compact expert-major rows, so padding
+// and dropped slots cost nothing.
+//
+//   D[r, n] = sum_k T[r, k] * W[e, n, k]        r in expert e's rows, n < Nw
+//
+// T ("token rows": x_gathered or the hidden activations) is [rows, K] and W is
+// [E, Nw, K]; both are K-major, which is what tcgen05 reads without transposes.
+//
+// Two tile orientations:
+//   - prefill (SWAP = false): the MMA's M = 128 token rows, N = BN weight rows;
+//   - decode  (SWAP = true):  M = 128 weight rows, N = up to BN tokens of one
+//     expert, so a 64-token batch still streams each weight tile once through
+//     a full-height MMA.
+// Work units are (expert, M tile, N tile, K split), enumerated from the
+// device-side counts by every CTA identically, and dealt round-robin.
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep
+// shared-memory ring; warp 1 owns the tensor memory and its lane 0 issues the
+// MMAs (4 x K=16 per 64-wide K block) and commits; warps 2-5 drain finished
+// accumulators (tcgen05.ld 32x32b: warp w reads TMEM lanes 32*(w%4)..+31),
+// apply ReLU, convert and store.  Two accumulator buffers let the epilogue of
+// one unit overlap the MMAs of the next.  Every wait is bounded in time: on
+// expiry the kernel records ST_TIMEOUT, lets in-flight copies and MMAs land,
+// frees its tensor memory and exits.
+#include "common.cuh"
+#include "internal.h"
+
+#include <cudaTypedefs.h>
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;       // MMA M
+constexpr int kBK = 64;        // K elements per stage (128 bytes of bf16 = one swizzle row)
+constexpr int kThreads = 192;
+
+enum { EPI_BF16 = 0, EPI_BF16_RELU = 1, EPI_F32 = 2 };
+
+struct TcArgs {
+    const int32_t *offsets;
+    const int32_t *counts;
+    int E, Nw, K, splits;
+    void *out;
+    int64_t ldo;           // elements per output row
+    int64_t split_stride;  // elements between K-split partial buffers (EPI_F32)
+    uint32_t *status;
+    uint64_t timeout_ns;
+};
+
+template <int BN>
+__host__ __device__ constexpr uint32_t tmem_cols() {
+    return 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+}
+
+struct Unit {
+    int e;
+    int tok0;     // first token row of the unit inside expert e
+    int w0;       // first weight row of the unit
+    int kb0, kb1; // K blocks [kb0, kb1)
+    int split;
+    int n_valid;  // valid columns of the MMA's N dimension
+};
+
+template <int BN, bool SWAP>
+__device__ __forceinline__ Unit decode_unit(int u, const int32_t *pre, const int32_t *cnt, int E,
+                                            int Nw, int splits, int kb_total) {
+    int lo = 0, hi = E;  // pre[lo] <= u < pre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] <= u) lo = mid; else hi = mid;
+    }
+    Unit t;
+    t.e = lo;
+    int r = u - pre[lo];
+    t.split = r % splits;
+    r /= splits;
+    const int c = cnt[lo];
+    if (!SWAP) {
+        const int mt = (c + kBM - 1) / kBM;
+        const int m = r % mt, n = r / mt;
+        t.tok0 = m * kBM;
+        t.w0 = n * BN;
+        t.n_valid = min(BN, Nw - t.w0);
+    } else {
+        const int tt = (c + BN - 1) / BN;
+        const int m = r / tt, n = r % tt;
+        t.w0 = m * kBM;
+        t.tok0 = n * BN;
+        t.n_valid = min(BN, c - t.tok0);
+    }
+    t.kb0 = static_cast<int>(static_cast<int64_t>(t.split) * kb_total / splits);
+    t.kb1 = static_cast<int>(static_cast<int64_t>(t.split + 1) * kb_total / splits);
+    return t;
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_timer_ns() - t0 > timeout_ns) return false;
+    return true;
+}
+
+template <int BN, bool SWAP, int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
+               const TcArgs args) {
+    constexpr uint32_t A_BYTES = kBM * kBK * 2;
+    constexpr uint32_t B_BYTES = BN * kBK * 2;
+    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+    __shared__ uint32_t tmem_holder;
+    __shared__ int32_t pre_s[257];
+    __shared__ int32_t cnt_s[256];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E, Nw = args.Nw, splits = args.splits;
+    const int kb_total = (args.K + kBK - 1) / kBK;
+    uint32_t *status = args.status;
+    const uint64_t tmo = args.timeout_ns;
+
+    const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    const uint32_t full0 = smem_u32(&bars[0]);
+    const uint32_t empty0 = smem_u32(&bars[STAGES]);
+    const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
+    const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            pre_s[e] = run;
+            const int c = cnt_s[e];
+            const int units = SWAP ? ((Nw + kBM - 1) / kBM) * ((c + BN - 1) / BN)
+                                   : ((c + kBM - 1) / kBM) * ((Nw + BN - 1) / BN);
+            run += units * splits;
+        }
+        pre_s[E] = run;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(tfull0, 1);
+        mbar_init(tfull0 + 8, 1);
+        mbar_init(tempty0, 4);
+        mbar_init(tempty0 + 8, 4);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_tok);
+        tma_prefetch_desc(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_holder;
+    const int total_units = pre_s[E];
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int issued = 0;
+            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+                const Unit t = decode_unit<BN, SWAP>(u, pre_s, cnt_s, E, Nw, splits, kb_total);
+                const int tok_row = args.offsets[t.e] + t.tok0;
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                    if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full0 + 8 * stage;
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const int kx = kb * kBK;
+                    if (!SWAP) {
+                        tma_load_2d(sa, &tm_tok, fb, kx, tok_row);
+                        tma_load_3d(sa + A_BYTES, &tm_w, fb, kx, t.w0, t.e);
+                    } else {
+                        tma_load_3d(sa, &tm_w, fb, kx, t.w0, t.e);
+                        tma_load_2d(sa + A_BYTES, &tm_tok, fb, kx, tok_row);
+                    }
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let copies already in flight land before the CTA can exit
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && i < issued; ++i) {
+                    if (st == 0) {
+                        st = STAGES - 1;
+                        ph ^= 1u;
+                    } else {
+                        --st;
+                    }
+                    wait_drain(full0 + 8 * st, ph, tmo);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, any = false;
+            int local = 0;
+            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+                const Unit t = decode_unit<BN, SWAP>(u, pre_s, cnt_s, E, Nw, splits, kb_total);
+                const int acc = local & 1;
+                const uint32_t acc_phase = (local >> 1) & 1;
+                if (!mbar_wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, status, tmo, 2)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                const int n_mma = (t.n_valid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
+                    if (!mbar_wait_bounded(full0 + 8 * stage, phase, status, tmo, 3)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint64_t ad = smem_desc_sw128(sa);
+                    const uint64_t bd = smem_desc_sw128(sa + A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        // +32 bytes along K inside the 128-byte swizzled row = +2 in the
+                        // descriptor's (address >> 4) field
+                        umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc,
+                                  (kb > t.kb0 || kk > 0) ? 1u : 0u);
+                    }
+                    any = true;
+                    umma_commit(empty0 + 8 * stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(tfull0 + 8 * acc);
+                ++local;
+            }
+            if (!ok && any) {
+                umma_commit(drain);
+                wait_drain(drain, 0, tmo);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+            const Unit t = decode_unit<BN, SWAP>(u, pre_s, cnt_s, E, Nw, splits, kb_total);
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            const bool mine = mbar_wait_bounded(tfull0 + 8 * acc, acc_phase, status, tmo, 4);
+            if (!__all_sync(0xffffffffu, mine)) break;
+            tc_fence_after();
+            const int cnt = cnt_s[t.e];
+            const int64_t row_base = args.offsets[t.e];
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * BN);
+            const int chunks = (t.n_valid + 31) >> 5;
+            for (int c = 0; c < chunks; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_wait_ld();
+                if (EPI == EPI_BF16_RELU) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
+                }
+                if (!SWAP) {
+                    const bool rv = t.tok0 + row_in_tile < cnt;
+                    const int64_t grow = row_base + t.tok0 + row_in_tile;
+                    const int col0 = t.w0 + c * 32;
+                    if (EPI == EPI_F32) {
+                        float *o = static_cast<float *>(args.out) + t.split * args.split_stride +
+                                   grow * args.ldo;
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            const int col = col0 + 4 * g;
+                            if (rv && col < Nw)
+                                *reinterpret_cast<float4 *>(o + col) =
+                                    make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                                __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+                        }
+                    } else {
+                        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = col0 + 8 * g;
+                            if (rv && col < Nw) {
+                                uint4 v;
+                                __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    h[i] = __floats2bfloat162_rn(__uint_as_float(r[8 * g + 2 * i]),
+                                                                 __uint_as_float(r[8 * g + 2 * i + 1]));
+                                *reinterpret_cast<uint4 *>(o + col) = v;
+                            }
+                        }
+                    }
+                } else {
+                    const int w = t.w0 + row_in_tile;
+                    if (w < Nw) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int tok = t.tok0 + c * 32 + i;
+                            if (tok < cnt) {
+                                const int64_t grow = row_base + tok;
+                                if (EPI == EPI_F32) {
+                                    static_cast<float *>(args.out)[t.split * args.split_stride +
+                                                                   grow * args.ldo + w] =
+                                        __uint_as_float(r[i]);
+                                } else {
+                                    static_cast<__nv_bfloat16 *>(args.out)[grow * args.ldo + w] =
+                                        __float2bfloat16_rn(__uint_as_float(r[i]));
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+            ++local;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bf16 [rows, K] K-major, box = 64 (K) x box_rows, 128-byte swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, int64_t rows, int K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [E, Nw, K] K-major, box = 64 (K) x box_rows x 1, 128-byte swizzle.
+bool make_map_3d(CUtensorMap *m, const void *base, int E, int Nw, int K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(Nw),
+                          static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(K) * 2 * Nw};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWAP, int EPI, int STAGES>
+cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
+                      const int32_t *offsets, const int32_t *counts, int splits, void *out,
+                      int64_t ldo, int64_t split_stride, uint32_t *status, uint64_t timeout_ns,
+                      int grid, cudaStream_t s) {
+    CUtensorMap tm_tok, tm_w;
+    if (!make_map_2d(&tm_tok, tok, tok_rows, K, SWAP ? BN : kBM)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tm_w, W, E, Nw, K, SWAP ? kBM : BN)) return cudaErrorInvalidValue;
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024;
+    auto kern = tc_gemm_kernel<BN, SWAP, EPI, STAGES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns};
+    kern<<<grid, kThreads, smem, s>>>(tm_tok, tm_w, a);
+    return cudaGetLastError();
+}
+
+// Sum of K-split fp32 partials into dtype rows, in split order.
+__global__ void __launch_bounds__(256)
+reduce_parts_kernel(const float *__restrict__ parts, int nparts, int64_t part_stride,
+                    const int32_t *__restrict__ offsets, int E, int d,
+                    __nv_bfloat16 *__restrict__ out) {
+    const int64_t rows = offsets[E];
+    const int64_t total = rows * (d / 4);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float4 a = reinterpret_cast<const float4 *>(parts)[i];
+        for (int p = 1; p < nparts; ++p) {
+            const float4 b = reinterpret_cast<const float4 *>(parts + p * part_stride)[i];
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(out) + 2 * i;
+        o[0] = __floats2bfloat162_rn(a.x, a.y);
+        o[1] = __floats2bfloat162_rn(a.z, a.w);
+    }
+}
+
+}  // namespace
+
+TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
+    TcPlan p{};
+    p.decode = rows <= 256;
+    p.splits_down = 1;
+    if (p.decode) {
+        const int64_t units = static_cast<int64_t>(E) * ((d + kBM - 1) / kBM);
+        const int kb_total = (d_ff + kBK - 1) / kBK;
+        int s = static_cast<int>((6LL * num_sms + units - 1) / units);
+        if (s > 8) s = 8;
+        if (s > kb_total) s = kb_total;
+        if (s < 1) s = 1;
+        p.splits_down = s;
+    }
+    return p;
+}
+
+size_t tc_ffn_ws_bytes(int64_t rows, int d, int d_ff, int E, int num_sms) {
+    const TcPlan p = plan_tc_ffn(rows, d, d_ff, E, num_sms);
+    size_t b = align_up(static_cast<size_t>(rows) * d_ff * 2, 256);  // hidden activations
+    if (p.decode) b += align_up(static_cast<size_t>(p.splits_down) * rows * d * 4, 256);
+    return b;
+}
+
+cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t *counts,
+                          const void *W_up, const void *W_down, int64_t rows, int d, int d_ff,
+                          int E, void *out, void *H, float *parts, bool combine_reads_parts,
+                          uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
+                          TcPlan *plan_out) {
+    const TcPlan p = plan_tc_ffn(rows, d, d_ff, E, num_sms);
+    if (plan_out) *plan_out = p;
+    cudaError_t e;
+    if (!p.decode) {
+        e = launch_tc<256, false, EPI_BF16_RELU, 4>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H,
+                                                    d_ff, 0, status, timeout_ns, num_sms, s);
+        if (e != cudaSuccess) return e;
+        return launch_tc<256, false, EPI_BF16, 4>(H, rows, W_down, E, d, d_ff, offsets, counts, 1, out,
+                                                  d, 0, status, timeout_ns, num_sms, s);
+    }
+    e = launch_tc<64, true, EPI_BF16_RELU, 8>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H, d_ff,
+                                              0, status, timeout_ns, num_sms, s);
+    if (e != cudaSuccess) return e;
+    const int64_t pstride = rows * static_cast<int64_t>(d);
+    e = launch_tc<64, true, EPI_F32, 8>(H, rows, W_down, E, d, d_ff, offsets, counts, p.splits_down,
+                                        parts, d, pstride, status, timeout_ns, num_sms, s);
+    if (e != cudaSuccess || combine_reads_parts) return e;
+    const int64_t total = rows * (d / 4);
+    const int blocks = static_cast<int>((total + 255) / 256 < 4 * num_sms ? (total + 255) / 256 : 4 * num_sms);
+    reduce_parts_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(parts, p.splits_down, pstride, offsets, E, d,
+                                                                static_cast<__nv_bfloat16 *>(out));
+    return cudaGetLastError();
+}
+
+// Diagnostic: one CTA waits on a barrier that nothing completes.
+__global__ void wait_timeout_kernel(uint32_t *status, uint64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(b, 0, status, timeout_ns, 9);
+    __syncthreads();
+}
+
+cudaError_t launch_wait_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s) {
+    wait_timeout_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

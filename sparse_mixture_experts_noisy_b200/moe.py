@@ -1,0 +1,266 @@
+"""Python binding of libmoe.so (include/moe.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; torch provides
+device memory and the stream.  There is no fallback: if the library is not
+built, or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+                4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
+
+EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch",
+           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
+           "moe_forward", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmoe.so and declare its signatures.  Raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(f"libmoe.so not built at {path}; run `python -m "
+                              "sparse_mixture_experts_noisy_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        P, I, I64, U32, F, D, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                                    ctypes.c_float, ctypes.c_double, ctypes.c_size_t)
+        sig = {
+            "moe_capacity": (I64, [I64, I, I, D]),
+            "moe_gathered_rows": (I64, [I64, I, I, D]),
+            "moe_route": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P]),
+            "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
+            "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
+            "moe_expert_ffn_workspace_size": (SZ, [I64, I, I, I, I]),
+            "moe_expert_ffn": (I, [P, P, P, P, P, I, I64, I, I, I, P, P, SZ, P]),
+            "moe_combine": (I, [P, P, P, P, P, I, I64, I, I, P, P]),
+            "moe_workspace_size": (SZ, [I64, I, I, I, I, D, I]),
+            "moe_forward": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_check_status": (I, [P, P, ctypes.POINTER(U32)]),
+            "moe_debug_wait_timeout": (I, [U32, P, SZ, P]),
+            "moe_num_sms": (I, []),
+            "moe_last_error": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+        return L
+
+
+def _check(code: int):
+    if code != 0:
+        raise MoeError(code, load_library().moe_last_error().decode())
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"storage type must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _cf(cf) -> float:
+    return math.inf if cf is None else float(cf)
+
+
+def capacity(N: int, E: int, k: int, cf) -> int:
+    return int(load_library().moe_capacity(N, E, k, _cf(cf)))
+
+
+def gathered_rows(N: int, E: int, k: int, cf) -> int:
+    return int(load_library().moe_gathered_rows(N, E, k, _cf(cf)))
+
+
+def num_sms() -> int:
+    return int(load_library().moe_num_sms())
+
+
+def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stream=None):
+    """-> (topk_idx [N,k] int32, gates [N,k] fp32, logits [N,E] fp32 or None)."""
+    L = load_library()
+    for t, n in ((x, "x"), (W_g, "W_g"), (b_g, "b_g"), (noise, "noise")):
+        _cuda(t, n)
+    N, d = x.shape
+    E = W_g.shape[0]
+    dev = x.device
+    topk = torch.empty((N, k), dtype=torch.int32, device=dev)
+    gates = torch.empty((N, k), dtype=torch.float32, device=dev)
+    logits = torch.empty((N, E), dtype=torch.float32, device=dev) if want_logits else None
+    _check(L.moe_route(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, k,
+                       _p(logits), _p(topk), _p(gates), _stream(stream)))
+    return topk, gates, logits
+
+
+def moe_dispatch(topk_idx, x, E, cf, stream=None):
+    """-> dict(slot, counts, offsets, x_gathered, rows, C)."""
+    L = load_library()
+    _cuda(topk_idx, "topk_idx")
+    _cuda(x, "x")
+    N, d = x.shape
+    k = topk_idx.shape[1]
+    dev = x.device
+    rows = L.moe_gathered_rows(N, E, k, _cf(cf))
+    if rows < 0:
+        raise MoeError(1, "invalid capacity arguments")
+    slot = torch.empty((N, k), dtype=torch.int32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    xg = torch.empty((rows, d), dtype=x.dtype, device=dev)
+    wsb = L.moe_dispatch_workspace_size(N, E, k)
+    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    _check(L.moe_dispatch(_p(topk_idx), _p(x), _dt(x), N, d, E, k, _cf(cf), _p(slot), _p(counts),
+                          _p(offsets), _p(xg), _p(ws), ws.numel(), _stream(stream)))
+    return dict(slot=slot, counts=counts, offsets=offsets, x_gathered=xg, rows=rows,
+                C=capacity(N, E, k, cf))
+
+
+def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=None, out=None):
+    """-> out_gathered [rows, d] (rows outside the kept ranges unspecified)."""
+    L = load_library()
+    for t, n in ((x_gathered, "x_gathered"), (offsets, "offsets"), (counts, "counts"), (W_up, "W_up"),
+                 (W_down, "W_down")):
+        _cuda(t, n)
+    rows, d = x_gathered.shape
+    E, d_ff, _ = W_up.shape
+    dt = _dt(x_gathered)
+    wsb = L.moe_expert_ffn_workspace_size(rows, d, E, d_ff, dt)
+    if ws is None:
+        ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=x_gathered.device)
+    if out is None:
+        out = torch.empty((rows, d), dtype=x_gathered.dtype, device=x_gathered.device)
+    _check(L.moe_expert_ffn(_p(x_gathered), _p(offsets), _p(counts), _p(W_up), _p(W_down), dt, rows, d,
+                            d_ff, E, _p(out), _p(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_combine(out_gathered, slot, topk_idx, offsets, gates, stream=None, y=None):
+    """-> y [N, d]."""
+    L = load_library()
+    N, k = slot.shape
+    d = out_gathered.shape[1]
+    if y is None:
+        y = torch.empty((N, d), dtype=out_gathered.dtype, device=out_gathered.device)
+    _check(L.moe_combine(_p(out_gathered), _p(slot), _p(topk_idx), _p(offsets), _p(gates),
+                         _dt(out_gathered), N, d, k, _p(y), _stream(stream)))
+    return y
+
+
+def workspace_size(N, d, E, d_ff, k, cf, dtype) -> int:
+    dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    return int(load_library().moe_workspace_size(N, d, E, d_ff, k, _cf(cf), dt))
+
+
+def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=None, ws=None,
+                intermediates=False, stream=None):
+    """The whole layer.  -> y, or (y, dict of logits/topk_idx/gates/slot/counts)."""
+    L = load_library()
+    for t, n in ((x, "x"), (W_g, "W_g"), (W_up, "W_up"), (W_down, "W_down"), (b_g, "b_g"),
+                 (noise, "noise")):
+        _cuda(t, n)
+    N, d = x.shape
+    E, d_ff, _ = W_up.shape
+    dev = x.device
+    wsb = workspace_size(N, d, E, d_ff, k, cf, x.dtype)
+    if wsb == 0:
+        raise MoeError(1, "invalid layer arguments")
+    if ws is None:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    if y is None:
+        y = torch.empty((N, d), dtype=x.dtype, device=dev)
+    inter = None
+    if intermediates:
+        inter = dict(logits=torch.empty((N, E), dtype=torch.float32, device=dev),
+                     topk_idx=torch.empty((N, k), dtype=torch.int32, device=dev),
+                     gates=torch.empty((N, k), dtype=torch.float32, device=dev),
+                     slot=torch.empty((N, k), dtype=torch.int32, device=dev),
+                     counts=torch.empty(E, dtype=torch.int32, device=dev))
+    g = (lambda n: _p(inter[n])) if inter else (lambda n: None)
+    _check(L.moe_forward(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, d_ff, k,
+                         _cf(cf), _p(W_up), _p(W_down), _p(y), g("logits"), g("topk_idx"), g("gates"),
+                         g("slot"), g("counts"), _p(ws), ws.numel(), _stream(stream)))
+    return (y, inter) if intermediates else y
+
+
+def check_status(ws, stream=None):
+    """Synchronise and read/clear a workspace's status word -> (code, raw word)."""
+    L = load_library()
+    word = ctypes.c_uint32(0)
+    code = L.moe_check_status(_p(ws), _stream(stream), ctypes.byref(word))
+    return int(code), int(word.value)
+
+
+def debug_wait_timeout(timeout_us: int, ws, stream=None):
+    _check(load_library().moe_debug_wait_timeout(int(timeout_us), _p(ws), ws.numel(), _stream(stream)))
+
+
+class MoELayer:
+    """Weights resident on the device plus a reusable workspace; __call__ runs
+    moe_forward on the current stream without allocating."""
+
+    def __init__(self, W_g, W_up, W_down, k, cf, b_g=None, sigma=0.0, max_tokens=None):
+        self.W_g, self.W_up, self.W_down, self.b_g = W_g, W_up, W_down, b_g
+        self.k, self.cf, self.sigma = int(k), cf, float(sigma)
+        self.E, self.d_ff, self.d = W_up.shape
+        self._ws = None
+        self._ws_tokens = -1
+        if max_tokens is not None:
+            self._reserve(max_tokens, W_up.dtype)
+
+    def _reserve(self, N, dtype):
+        need = workspace_size(N, self.d, self.E, self.d_ff, self.k, self.cf, dtype)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.W_up.device)
+        self._ws_tokens = N
+
+    @property
+    def workspace(self):
+        return self._ws
+
+    def __call__(self, x, noise=None, y=None, stream=None):
+        if self._ws is None or x.shape[0] != self._ws_tokens:
+            self._reserve(x.shape[0], x.dtype)
+        return moe_forward(x, self.W_g, self.W_up, self.W_down, self.k, self.cf, b_g=self.b_g,
+                           noise=noise, sigma=self.sigma, y=y, ws=self._ws, stream=stream)

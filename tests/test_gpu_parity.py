@@ -1,0 +1,164 @@
+"""CUDA path against the CPU oracle, element by element (needs a B200).
+
+Routing (top-k indices, slots, counts, the drop set) must match the oracle
+bit-exactly when the oracle replays the GPU's fp32 logits; gates within 2e-6;
+the layer output within max|y - y_oracle| / max|y_oracle| <= 1e-5 (fp32) or
+2e-2 (bf16)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_mixture_experts_noisy_b200 import moe
+from sparse_mixture_experts_noisy_b200.synth import WORKLOADS, Workload, F32, BF16
+from tests.gpu_util import Case, TOL, check_routing, rel_err, require_gpu, to_host_bits, values
+
+pytestmark = pytest.mark.gpu
+
+W = WORKLOADS
+SMALL = {
+    # several M tiles per expert with a ragged tail, ragged N tile (384 = 256 + 128)
+    "nano_small": W["nano"].with_(N=1000, d=256, d_ff=384, wg_std=1 / 16),
+    # router bias +1 on expert 0 overflows its capacity: drops
+    "mixtral_small": W["mixtral"].with_(N=1536, d=512, d_ff=1024),
+    # 64 experts, k = 6, supplied noise, d_ff not a multiple of the N tile
+    "fine_small": W["fine"].with_(N=2048, d=256, d_ff=176),
+    # few tokens per expert: weight-stationary tiles and split-K down projection
+    "decode_small": W["decode"].with_(N=64, d=512, d_ff=1024),
+    "decode_ragged": W["decode"].with_(N=37, d=256, d_ff=320, k=3),
+    # fp32 storage: CUDA-core FFN, drops, ragged everything
+    "f32_drops": Workload("f32_drops", F32, N=300, d=40, E=6, d_ff=50, k=3, sigma=0.5, cf=0.8,
+                          w_std=0.3, wg_std=0.3),
+    # bf16 rows that are not 16-byte multiples: CUDA-core FFN in bf16
+    "bf16_unaligned": Workload("bf16_unaligned", BF16, N=200, d=36, E=5, d_ff=20, k=2, sigma=0.0, cf=1.0,
+                               w_std=0.2, wg_std=0.3),
+    "switch_k1": W["nano"].with_(N=700, d=128, d_ff=256, k=1, cf=1.0, wg_std=0.1),
+    "dense_k_eq_E": W["nano"].with_(N=300, d=128, d_ff=128, E=4, k=4, cf=math.inf, wg_std=0.1),
+    "single_expert": W["nano"].with_(N=257, d=64, d_ff=64, E=1, k=1, cf=1.0, wg_std=0.1),
+    "many_drops": W["nano"].with_(N=512, d=128, d_ff=256, cf=0.05, wg_std=0.1),
+    "one_token": W["nano"].with_(N=1, d=64, d_ff=128, wg_std=0.1),
+    "toy": W["toy"],
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check_case(wl, seed=0, tokens=None):
+    case = Case(wl, seed)
+    y, inter = case.forward()
+    torch.cuda.synchronize()
+    lg, idx, g, slot, counts = check_routing(case, inter)
+    ref = case.oracle_from_logits(lg, tokens)
+    yh = values(to_host_bits(y))
+    if tokens is not None:
+        yh = yh[tokens]
+    err = rel_err(yh, ref["y"])
+    assert err <= TOL[wl.dtype], f"{wl.name}: output error {err:.3g} > {TOL[wl.dtype]}"
+    # tokens whose every choice was dropped get exact zero rows
+    dropped = np.all(slot < 0, axis=1)
+    if dropped.any():
+        assert np.all(values(to_host_bits(y))[dropped] == 0.0)
+    return case, y, inter, err
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_small(name):
+    _check_case(SMALL[name])
+
+
+def test_many_drops_really_drops():
+    case, y, inter, _ = _check_case(SMALL["many_drops"])
+    slot = inter["slot"].cpu().numpy()
+    assert np.sum(slot < 0) > 0.5 * slot.size
+    assert np.any(np.all(slot < 0, axis=1))
+
+
+def test_empty_batch():
+    wl = W["nano"].with_(N=0, d=64, d_ff=128)
+    case = Case(wl)
+    y, inter = case.forward()
+    torch.cuda.synchronize()
+    assert y.shape == (0, 64)
+    assert inter["counts"].cpu().numpy().tolist() == [0] * wl.E
+
+
+def test_staged_calls_match_fused_forward():
+    """moe_route -> moe_dispatch -> moe_expert_ffn -> moe_combine gives the
+    fused result bit for bit; x_gathered rows are exact copies of x; every
+    expert-output row matches the oracle's expert FFN."""
+    wl = SMALL["mixtral_small"]
+    case = Case(wl, seed=5)
+    y_fused, inter = case.forward()
+    topk, gates, logits = moe.moe_route(case.x, case.W_g, wl.k, b_g=case.b_g, noise=case.noise,
+                                        sigma=wl.sigma)
+    d = moe.moe_dispatch(topk, case.x, wl.E, wl.cf)
+    out = moe.moe_expert_ffn(d["x_gathered"], d["offsets"], d["counts"], case.W_up, case.W_down)
+    y = moe.moe_combine(out, d["slot"], topk, d["offsets"], gates)
+    torch.cuda.synchronize()
+    assert torch.equal(logits, inter["logits"]) and torch.equal(topk, inter["topk_idx"])
+    assert torch.equal(gates, inter["gates"]) and torch.equal(d["slot"], inter["slot"])
+    assert torch.equal(y.view(torch.int16), y_fused.view(torch.int16))
+    slot = d["slot"].cpu().numpy()
+    offs = d["offsets"].cpu().numpy()
+    tk = topk.cpu().numpy()
+    xg = to_host_bits(d["x_gathered"])
+    og = values(to_host_bits(out))
+    x = case.inp.x
+    rng = np.random.default_rng(0)
+    checked = 0
+    for t in range(wl.N):
+        for j in range(wl.k):
+            if slot[t, j] < 0:
+                continue
+            r = offs[tk[t, j]] + slot[t, j]
+            assert np.array_equal(xg[r], x[t])
+            if rng.random() < 0.05:
+                _, o = oracle.expert_ffn(x, case.inp.W_up, case.inp.W_down, t, tk[t, j])
+                assert rel_err(og[r], o) <= TOL[wl.dtype]
+                checked += 1
+    assert checked > 10
+    assert offs[-1] == int(d["counts"].sum())
+
+
+def test_deterministic():
+    wl = SMALL["fine_small"]
+    case = Case(wl, seed=2)
+    y1, i1 = case.forward()
+    y2, i2 = case.forward()
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    for key in i1:
+        assert torch.equal(i1[key], i2[key])
+
+
+def test_sigma_zero_equals_no_noise():
+    wl = SMALL["fine_small"]
+    case = Case(wl, seed=1)
+    y_a = moe.moe_forward(case.x, case.W_g, case.W_up, case.W_down, wl.k, wl.cf, noise=case.noise, sigma=0.0)
+    y_b = moe.moe_forward(case.x, case.W_g, case.W_up, case.W_down, wl.k, wl.cf, noise=None, sigma=0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(y_a.view(torch.int16), y_b.view(torch.int16))
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    moe.debug_wait_timeout(20000, ws)
+    code, word = moe.check_status(ws)
+    assert code == 6 and (word & 1)
+    code, word = moe.check_status(ws)      # cleared
+    assert code == 0 and word == 0
+    _check_case(SMALL["decode_small"])    # the context is still usable
+
+
+def test_status_clean_after_forward():
+    wl = SMALL["nano_small"]
+    case = Case(wl)
+    layer = moe.MoELayer(case.W_g, case.W_up, case.W_down, wl.k, wl.cf, b_g=case.b_g, sigma=wl.sigma)
+    layer(case.x, noise=case.noise)
+    code, word = moe.check_status(layer.workspace)
+    assert code == 0 and word == 0
