@@ -34,7 +34,6 @@ METRIC = "MoE layer tokens/sec at 1 B200; % of bf16 tensor peak (prefill) / HBM 
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
-KERNELS_PER_FORWARD = 7  # route, hist, scan, assign+gather, up GEMM, down GEMM, combine
 
 
 def parse_args(argv=None):
@@ -310,12 +309,14 @@ def time_steps(fn, steps, torch, flush=None):
 
 
 def measure_layer(wl, inp_dev, steps, warmup, dist, torch, moe, flush_needed):
+    """moe_forward replayed from a CUDA graph (one graph launch per step)."""
     x, W_g, b_g, noise, W_up, W_down = inp_dev
     layer = moe.MoELayer(W_g, W_up, W_down, wl.k, wl.cf, b_g=b_g, sigma=wl.sigma, max_tokens=wl.N)
-    y = torch.empty_like(x)
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=x.device) if flush_needed else None
     flush = (lambda: flush_buf.fill_(1)) if flush_needed else None
-    run = lambda: layer(x, noise=noise, y=y)  # noqa: E731
+    graphed = moe.GraphedForward(layer, x, noise)
+    y = graphed.y
+    run = graphed.replay
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
@@ -329,7 +330,7 @@ def measure_layer(wl, inp_dev, steps, warmup, dist, torch, moe, flush_needed):
     code, word = moe.check_status(layer.workspace)
     if code != 0:
         raise RuntimeError(f"kernel status {code} (0x{word:08x}) after the timed region")
-    return layer, y, sec, clk.summary()
+    return graphed, y, sec, clk.summary()
 
 
 def measure_ffn(wl, inp_dev, steps, torch, moe):
@@ -353,24 +354,22 @@ def measure_ffn(wl, inp_dev, steps, torch, moe):
     return sec / steps, counts
 
 
-def measure_e2e(layer, wl, inp, steps, torch, moe):
-    """Through the public API with host buffers: pinned x (and eps) copied in,
-    moe_forward, y copied out, every step."""
-    x_h = torch.from_numpy(inp.x.view(np.int16) if inp.x.dtype == np.uint16 else inp.x).pin_memory()
-    n_h = torch.from_numpy(inp.noise).pin_memory() if inp.noise is not None else None
-    x_d = torch.empty(x_h.shape, dtype=x_h.dtype, device="cuda")
-    n_d = torch.empty(n_h.shape, dtype=n_h.dtype, device="cuda") if n_h is not None else None
-    y_d = torch.empty(x_h.shape, dtype=x_h.dtype, device="cuda")
-    y_h = torch.empty(x_h.shape, dtype=x_h.dtype).pin_memory()
+def measure_e2e(graphed, wl, inp, steps, torch, moe):
+    """Through the public API with host buffers: pinned x (and eps) copied into
+    the graphed forward's input buffers, the forward replayed, y copied back to
+    pinned host memory, every step."""
     bf = inp.x.dtype == np.uint16
+    x_h = torch.from_numpy(inp.x.view(np.int16) if bf else inp.x).pin_memory()
+    x_h = x_h.view(torch.bfloat16) if bf else x_h
+    n_h = torch.from_numpy(inp.noise).pin_memory() if inp.noise is not None else None
+    y_h = torch.empty(x_h.shape, dtype=x_h.dtype).pin_memory()
 
     def step():
-        x_d.copy_(x_h, non_blocking=True)
-        if n_d is not None:
-            n_d.copy_(n_h, non_blocking=True)
-        xv = x_d.view(torch.bfloat16) if bf else x_d
-        layer(xv, noise=n_d, y=y_d.view(torch.bfloat16) if bf else y_d)
-        y_h.copy_(y_d, non_blocking=True)
+        graphed.x.copy_(x_h, non_blocking=True)
+        if n_h is not None:
+            graphed.noise.copy_(n_h, non_blocking=True)
+        graphed.replay()
+        y_h.copy_(graphed.y, non_blocking=True)
 
     for _ in range(3):
         step()
@@ -445,7 +444,7 @@ def run_ours(args):
             "roofline": roof,
             "e2e": {"value": wl.N * dist.world / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "gpu_launches": moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) * args.steps,
             "clocks": clocks}
 
     # the decode-shaped workload shares the weights' shapes and seeds with the
@@ -472,7 +471,8 @@ def run_ours(args):
                                         "whole_layer_frac": layer_bytes / (dmax / dsteps) / 1e9 / peaks["hbm_gbs"],
                                         "whole_layer_frac_of_8tbs": layer_bytes / (dmax / dsteps) / 8e12}),
             "clocks": dclk}
-        line["gpu_launches"] += KERNELS_PER_FORWARD * dsteps
+        line["gpu_launches"] += moe.forward_launches(dwl.N, dwl.d, dwl.E, dwl.d_ff, dwl.k, dwl.cf,
+                                                     ddev[0].dtype) * dsteps
 
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cores = cpu_cores()

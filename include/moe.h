@@ -175,6 +175,11 @@ MOE_API moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, co
                        int32_t *slot_out, int32_t *counts_out,
                        void *ws, size_t ws_bytes, void *stream);
 
+/* Number of kernels one moe_forward call with these arguments launches on its
+ * stream (0 for N = 0, -1 for invalid arguments).  Useful to size CUDA-graph
+ * captures and to account for launches. */
+MOE_API int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronises `stream` and reads the status word at the start of a workspace

@@ -340,6 +340,13 @@ moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const floa
     return MOE_OK;
 }
 
+int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt) {
+    if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1 || moe_capacity(N, E, k, cf) < 0) return -1;
+    if (N == 0) return 0;
+    // router + dispatch passes + two expert GEMMs + combine
+    return 1 + moe::dispatch_launches(N, E, k) + 2 + 1;
+}
+
 moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {
     if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "ws must not be NULL");
     cudaStream_t s = static_cast<cudaStream_t>(stream);

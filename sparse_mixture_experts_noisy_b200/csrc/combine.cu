@@ -5,8 +5,9 @@
 // cb_weight @ exp_out: a dropped pair has weight 0, the kept ones keep their
 // gate, so a token whose choices were all dropped gets a zero row).
 // The dense [tokens, E*C] x [E*C, d] product of the slides is replaced by a
-// gather: one warp per token reads its k expert-output rows and accumulates
-// g * row in fp32, in choice order j = 0..k-1.
+// gather: a block takes one token at a time, each thread owns a chunk of its
+// output columns, reads that chunk of the token's k expert-output rows and
+// accumulates g * row in fp32, in choice order j = 0..k-1.
 //
 // The expert outputs are either rows of dtype T (one partial) or `parts`
 // fp32 partial sums over K-splits of the down projection, which are added in
@@ -17,8 +18,6 @@
 namespace moe {
 
 namespace {
-
-constexpr int kCombineWarps = 8;
 
 template <typename T, int VEC>
 struct Vec;
@@ -74,50 +73,54 @@ __device__ __forceinline__ void load_f32(const float *p, float (&v)[VEC]) {
 }
 
 template <typename T, int VEC>
-__global__ void __launch_bounds__(kCombineWarps * 32)
+__global__ void __launch_bounds__(256)
 combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, int nparts,
                int64_t part_stride, const int32_t *__restrict__ slot,
                const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
                const float *__restrict__ gates, int64_t N, int d, int k, int E,
                T *__restrict__ y) {
+    // a block takes tokens in turn; its threads split the token's columns into
+    // VEC-wide chunks; the token's k (row, gate) pairs are read once per block
     extern __shared__ int32_t c_smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int32_t *rows = c_smem + warp * 2 * k;                       // [k] source row or -1
-    float *g = reinterpret_cast<float *>(rows + k);              // [k]
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
-    if (t >= N) return;
-    for (int j = lane; j < k; j += 32) {
-        const int32_t sl = slot[t * k + j];
-        const int32_t e = topk_idx[t * k + j];
-        const bool ok = sl >= 0 && e >= 0 && e < E;
-        rows[j] = ok ? offsets[e] + sl : -1;
-        g[j] = ok ? gates[t * k + j] : 0.0f;
-    }
-    __syncwarp();
-    for (int c = lane * VEC; c < d; c += 32 * VEC) {
-        float acc[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int32_t r = rows[j];
-            if (r < 0) continue;
-            float o[VEC];
-            if (nparts == 0) {
-                Vec<T, VEC>::load(out_rows + static_cast<int64_t>(r) * d + c, o);
-            } else {
-                load_f32<VEC>(parts + static_cast<int64_t>(r) * d + c, o);
-                for (int p = 1; p < nparts; ++p) {
-                    float q[VEC];
-                    load_f32<VEC>(parts + p * part_stride + static_cast<int64_t>(r) * d + c, q);
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) o[v] += q[v];
-                }
-            }
-            const float gj = g[j];
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj, o[v], acc[v]);
+    int32_t *rows = c_smem;                                  // [k] source row or -1
+    float *g = reinterpret_cast<float *>(rows + k);          // [k]
+    const int chunks = d / VEC;
+    for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
+        for (int j = threadIdx.x; j < k; j += blockDim.x) {
+            const int32_t sl = slot[t * k + j];
+            const int32_t e = topk_idx[t * k + j];
+            const bool ok = sl >= 0 && e >= 0 && e < E;
+            rows[j] = ok ? offsets[e] + sl : -1;
+            g[j] = ok ? gates[t * k + j] : 0.0f;
         }
-        Vec<T, VEC>::store(y + t * d + c, acc);
+        __syncthreads();
+        for (int ch = threadIdx.x; ch < chunks; ch += blockDim.x) {
+            const int c = ch * VEC;
+            float acc[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = rows[j];
+                if (r < 0) continue;
+                float o[VEC];
+                if (nparts == 0) {
+                    Vec<T, VEC>::load(out_rows + static_cast<int64_t>(r) * d + c, o);
+                } else {
+                    load_f32<VEC>(parts + static_cast<int64_t>(r) * d + c, o);
+                    for (int p = 1; p < nparts; ++p) {
+                        float q[VEC];
+                        load_f32<VEC>(parts + p * part_stride + static_cast<int64_t>(r) * d + c, q);
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) o[v] += q[v];
+                    }
+                }
+                const float gj = g[j];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj, o[v], acc[v]);
+            }
+            Vec<T, VEC>::store(y + t * d + c, acc);
+        }
+        __syncthreads();
     }
 }
 
@@ -126,11 +129,16 @@ cudaError_t launch_combine_t(const void *out_rows, const float *parts, int npart
                              int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
                              const int32_t *offsets, const float *gates, int64_t N, int d, int k,
                              int E, void *y, cudaStream_t s) {
-    const int64_t blocks = (N + kCombineWarps - 1) / kCombineWarps;
-    const size_t smem = sizeof(int32_t) * 2 * static_cast<size_t>(k) * kCombineWarps;
-    combine_kernel<T, VEC><<<static_cast<unsigned>(blocks), kCombineWarps * 32, smem, s>>>(
-        static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets,
-        gates, N, d, k, E, static_cast<T *>(y));
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int chunks = d / VEC;
+    const int threads = chunks >= 256 ? 256 : (chunks >= 128 ? 128 : (chunks >= 64 ? 64 : 32));
+    int64_t blocks = N;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    const size_t smem = sizeof(int32_t) * 2 * static_cast<size_t>(k);
+    combine_kernel<T, VEC><<<static_cast<unsigned>(blocks), threads, smem, s>>>(
+        static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets, gates, N,
+        d, k, E, static_cast<T *>(y));
     return cudaGetLastError();
 }
 

@@ -13,8 +13,9 @@
 //              the total over all tokens;
 //   3. assign: place(t, j) = sum_{j' < j} total[j'][e] + prefix over earlier
 //              blocks + rank among earlier tokens of the same block (warp
-//              match + per-warp counts), then slot = place < C ? place : -1, and
-//              the kept rows are copied to x_gathered[offsets[e] + place].
+//              match + per-warp counts), then slot = place < C ? place : -1;
+//   4. gather: the kept rows are copied to x_gathered[offsets[e] + place].
+// Batches of at most 1024 tokens do passes 1-3 in one block.
 // No step depends on the order in which threads or blocks run.
 #include "common.cuh"
 #include "internal.h"
@@ -69,31 +70,17 @@ scan_kernel(int32_t *__restrict__ hist, int nblk, int E, int k, int32_t *__restr
     if (lane == 0) tot[pair] = carry;
 }
 
-__device__ __forceinline__ void copy_row(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
-                                         int64_t bytes, bool vec16, int lane) {
-    if (vec16) {
-        const uint4 *s = reinterpret_cast<const uint4 *>(src);
-        uint4 *d = reinterpret_cast<uint4 *>(dst);
-        for (int64_t i = lane; i < bytes / 16; i += 32) d[i] = s[i];
-    } else {
-        const uint16_t *s = reinterpret_cast<const uint16_t *>(src);
-        uint16_t *d = reinterpret_cast<uint16_t *>(dst);
-        for (int64_t i = lane; i < bytes / 2; i += 32) d[i] = s[i];
-    }
-}
-
+// Queue places and drops for one block of kDispatchTB tokens; block 0 also
+// publishes counts and offsets.  hist_excl/tot come from the scan.
 __global__ void __launch_bounds__(kDispatchTB)
-assign_kernel(const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ x, int64_t row_bytes,
-              bool vec16, int64_t N, int E, int k, int64_t C,
+assign_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int64_t C,
               const int32_t *__restrict__ hist_excl /* [nblk][k][E] */,
               const int32_t *__restrict__ tot /* [k][E] */, int32_t *__restrict__ slot,
-              int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
-              uint8_t *__restrict__ x_gathered) {
+              int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
     extern __shared__ int32_t a_smem[];
     int32_t *warp_cnt = a_smem;                                // [warps][E]
     int32_t *jrun = warp_cnt + kDispatchWarps * E;             // [E]  sum_{j' < j} tot[j'][e]
     int32_t *offs = jrun + E;                                  // [E + 1]
-    int32_t *rowmap = offs + E + 1;                            // [TB] destination row or -1
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchTB + tid;
@@ -134,36 +121,124 @@ assign_kernel(const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ 
         const int rank_in_warp = __popc(same & lt_mask);
         if (e >= 0 && rank_in_warp == 0) warp_cnt[warp * E + e] = __popc(same);
         __syncthreads();
-        int32_t r = -1;
         if (e >= 0) {
             int64_t place = static_cast<int64_t>(jrun[e]) +
                             hist_excl[(static_cast<int64_t>(blockIdx.x) * k + j) * E + e] + rank_in_warp;
             for (int w = 0; w < warp; ++w) place += warp_cnt[w * E + e];
-            const bool kept = place < C;
-            slot[t * k + j] = kept ? static_cast<int32_t>(place) : -1;
-            if (kept) r = offs[e] + static_cast<int32_t>(place);
+            slot[t * k + j] = place < C ? static_cast<int32_t>(place) : -1;
         } else if (t < N) {
             slot[t * k + j] = -1;
         }
-        rowmap[tid] = r;
         __syncthreads();
-        // copy the kept rows of this choice rank, one warp per row
-        for (int i = warp; i < kDispatchTB; i += kDispatchWarps) {
-            const int32_t dst = rowmap[i];
-            if (dst >= 0) {
-                const int64_t ts = static_cast<int64_t>(blockIdx.x) * kDispatchTB + i;
-                copy_row(x + ts * row_bytes, x_gathered + static_cast<int64_t>(dst) * row_bytes,
-                         row_bytes, vec16, lane);
-            }
-        }
         for (int ee = tid; ee < E; ee += blockDim.x) jrun[ee] += tot[j * E + ee];
         __syncthreads();
+    }
+}
+
+// The whole slot assignment for a batch of at most kSmallTB tokens in one
+// block: count per (j, e), then place each (t, j) in token order within its
+// choice rank (warp match + per-warp counts), as in the multi-block passes.
+constexpr int kSmallTB = 1024;
+constexpr int kSmallWarps = kSmallTB / 32;
+
+__global__ void __launch_bounds__(kSmallTB)
+dispatch_small_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int64_t C,
+                      int32_t *__restrict__ slot, int32_t *__restrict__ counts,
+                      int32_t *__restrict__ offsets) {
+    extern __shared__ int32_t s_smem[];
+    int32_t *tot = s_smem;                         // [k][E]
+    int32_t *warp_cnt = tot + k * E;               // [warps][E]
+    int32_t *jrun = warp_cnt + kSmallWarps * E;    // [E]
+    int32_t *offs = jrun + E;                      // [E + 1]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = tid;
+    for (int i = tid; i < k * E; i += blockDim.x) tot[i] = 0;
+    __syncthreads();
+    if (t < N)
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[t * k + j];
+            if (e >= 0 && e < E) atomicAdd(&tot[j * E + e], 1);
+        }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+        int64_t total = 0;
+        for (int j = 0; j < k; ++j) total += tot[j * E + e];
+        offs[e] = static_cast<int32_t>(total < C ? total : C);
+        jrun[e] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int32_t run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t c = offs[e];
+            offs[e] = run;
+            counts[e] = c;
+            offsets[e] = run;
+            run += c;
+        }
+        offs[E] = run;
+        offsets[E] = run;
+    }
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+        for (int i = tid; i < kSmallWarps * E; i += blockDim.x) warp_cnt[i] = 0;
+        __syncthreads();
+        int e = -1;
+        if (t < N) {
+            e = topk_idx[t * k + j];
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank_in_warp = __popc(same & lt_mask);
+        if (e >= 0 && rank_in_warp == 0) warp_cnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        if (e >= 0) {
+            int64_t place = static_cast<int64_t>(jrun[e]) + rank_in_warp;
+            for (int w = 0; w < warp; ++w) place += warp_cnt[w * E + e];
+            slot[t * k + j] = place < C ? static_cast<int32_t>(place) : -1;
+        } else if (t < N) {
+            slot[t * k + j] = -1;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += blockDim.x) jrun[ee] += tot[j * E + ee];
+        __syncthreads();
+    }
+}
+
+// x_gathered[offsets[e] + slot[t][j]] = x[t] for every kept (t, j): one thread
+// per (t, j, unit), units being 16 bytes (2 bytes when rows are not 16-byte
+// multiples), so even a handful of tokens spreads over the whole GPU.
+template <typename U>
+__global__ void __launch_bounds__(256)
+gather_kernel(const U *__restrict__ x, int64_t units_per_row, const int32_t *__restrict__ topk_idx,
+              const int32_t *__restrict__ slot, const int32_t *__restrict__ offsets, int64_t Nk, int k,
+              U *__restrict__ xg) {
+    const int64_t total = Nk * units_per_row;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t tj = i / units_per_row;
+        const int64_t c = i - tj * units_per_row;
+        const int32_t sl = slot[tj];
+        if (sl < 0) continue;
+        const int64_t row = static_cast<int64_t>(offsets[topk_idx[tj]]) + sl;
+        xg[row * units_per_row + c] = x[(tj / k) * units_per_row + c];
     }
 }
 
 }  // namespace
 
 int64_t dispatch_blocks(int64_t N) { return (N + kDispatchTB - 1) / kDispatchTB; }
+
+bool dispatch_single_block(int64_t N, int E, int k) {
+    const size_t small_smem = sizeof(int32_t) * (static_cast<size_t>(k) * E + kSmallWarps * E + E + E + 1);
+    return N <= kSmallTB && small_smem <= 48 * 1024;
+}
+
+int dispatch_launches(int64_t N, int E, int k) {
+    if (N == 0) return 0;
+    return dispatch_single_block(N, E, k) ? 2 : 4;
+}
 
 size_t dispatch_ws_bytes(int64_t N, int E, int k) {
     const int64_t nblk = dispatch_blocks(N);
@@ -175,28 +250,55 @@ size_t dispatch_ws_bytes(int64_t N, int E, int k) {
 cudaError_t launch_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N,
                             int d, int E, int k, int64_t C, int32_t *slot, int32_t *counts,
                             int32_t *offsets, void *x_gathered, void *ws, cudaStream_t s) {
-    const int64_t nblk = dispatch_blocks(N);
-    int32_t *hist = static_cast<int32_t *>(ws);
-    int32_t *tot = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) +
-                                               align_up(sizeof(int32_t) * static_cast<size_t>(nblk > 0 ? nblk : 1) * k * E, 256));
     if (N == 0) {
         cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
         if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
         return e;
     }
-    hist_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, sizeof(int32_t) * E, s>>>(topk_idx, N, E,
-                                                                                     k, hist);
-    const int pairs = k * E;
-    const int warps_per_block = 8;
-    scan_kernel<<<(pairs + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, s>>>(
-        hist, static_cast<int>(nblk), E, k, tot);
+    const size_t small_smem = sizeof(int32_t) * (static_cast<size_t>(k) * E + kSmallWarps * E + E + E + 1);
+    if (dispatch_single_block(N, E, k)) {
+        dispatch_small_kernel<<<1, kSmallTB, small_smem, s>>>(topk_idx, N, E, k, C, slot, counts, offsets);
+    } else {
+        const int64_t nblk = dispatch_blocks(N);
+        int32_t *hist = static_cast<int32_t *>(ws);
+        int32_t *tot = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) +
+                                                   align_up(sizeof(int32_t) * static_cast<size_t>(nblk) * k * E, 256));
+        hist_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, sizeof(int32_t) * E, s>>>(topk_idx, N, E,
+                                                                                         k, hist);
+        const int pairs = k * E;
+        const int warps_per_block = 8;
+        scan_kernel<<<(pairs + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, s>>>(
+            hist, static_cast<int>(nblk), E, k, tot);
+        const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kDispatchWarps) * E + E + E + 1);
+        assign_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, smem, s>>>(topk_idx, N, E, k, C, hist, tot,
+                                                                            slot, counts, offsets);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_gather(topk_idx, slot, offsets, x, elem_bytes, N, d, k, x_gathered, s);
+}
+
+cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const int32_t *offsets,
+                          const void *x, int elem_bytes, int64_t N, int d, int k, void *x_gathered,
+                          cudaStream_t s) {
     const int64_t row_bytes = static_cast<int64_t>(d) * elem_bytes;
     const bool vec16 = (row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
                        (reinterpret_cast<uintptr_t>(x_gathered) % 16 == 0);
-    const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kDispatchWarps) * E + E + E + 1 + kDispatchTB);
-    assign_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, smem, s>>>(
-        topk_idx, static_cast<const uint8_t *>(x), row_bytes, vec16, N, E, k, C, hist, tot, slot,
-        counts, offsets, static_cast<uint8_t *>(x_gathered));
+    const int64_t Nk = N * k;
+    const int64_t units = vec16 ? row_bytes / 16 : row_bytes / 2;
+    const int64_t total = Nk * units;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    if (blocks < 1) blocks = 1;
+    if (vec16)
+        gather_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            static_cast<const uint4 *>(x), units, topk_idx, slot, offsets, Nk, k, static_cast<uint4 *>(x_gathered));
+    else
+        gather_kernel<uint16_t><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            static_cast<const uint16_t *>(x), units, topk_idx, slot, offsets, Nk, k,
+            static_cast<uint16_t *>(x_gathered));
     return cudaGetLastError();
 }
 

@@ -17,10 +17,15 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
 
 // Dispatch (dispatch.cu).
 int64_t dispatch_blocks(int64_t N);
+bool dispatch_single_block(int64_t N, int E, int k);
+int dispatch_launches(int64_t N, int E, int k);  // kernels launch_dispatch issues
 size_t dispatch_ws_bytes(int64_t N, int E, int k);
 cudaError_t launch_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N,
                             int d, int E, int k, int64_t C, int32_t *slot, int32_t *counts,
                             int32_t *offsets, void *x_gathered, void *ws, cudaStream_t s);
+cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const int32_t *offsets,
+                          const void *x, int elem_bytes, int64_t N, int d, int k, void *x_gathered,
+                          cudaStream_t s);
 
 // Combine (combine.cu).  Either out_rows (dtype rows, nparts == 0) or nparts
 // fp32 partial buffers `part_stride` elements apart.

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 
 EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
-           "moe_forward", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
+           "moe_forward", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
 
 class MoeError(RuntimeError):
@@ -58,6 +58,7 @@ def load_library(path: str = LIB_PATH):
             "moe_combine": (I, [P, P, P, P, P, I, I64, I, I, P, P]),
             "moe_workspace_size": (SZ, [I64, I, I, I, I, D, I]),
             "moe_forward": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_forward_launches": (I, [I64, I, I, I, I, D, I]),
             "moe_check_status": (I, [P, P, ctypes.POINTER(U32)]),
             "moe_debug_wait_timeout": (I, [U32, P, SZ, P]),
             "moe_num_sms": (I, []),
@@ -193,6 +194,11 @@ def workspace_size(N, d, E, d_ff, k, cf, dtype) -> int:
     return int(load_library().moe_workspace_size(N, d, E, d_ff, k, _cf(cf), dt))
 
 
+def forward_launches(N, d, E, d_ff, k, cf, dtype) -> int:
+    dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
+    return int(load_library().moe_forward_launches(N, d, E, d_ff, k, _cf(cf), dt))
+
+
 def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=None, ws=None,
                 intermediates=False, stream=None):
     """The whole layer.  -> y, or (y, dict of logits/topk_idx/gates/slot/counts)."""
@@ -264,3 +270,33 @@ class MoELayer:
             self._reserve(x.shape[0], x.dtype)
         return moe_forward(x, self.W_g, self.W_up, self.W_down, self.k, self.cf, b_g=self.b_g,
                            noise=noise, sigma=self.sigma, y=y, ws=self._ws, stream=stream)
+
+
+class GraphedForward:
+    """moe_forward captured once in a CUDA graph over static buffers.
+
+    The library launches every kernel of the layer on the capturing stream and
+    allocates nothing, so the whole forward replays as one graph launch.  Copy
+    new inputs into `.x` (and `.noise`) before `replay()`; the output lands in
+    `.y`.  The graph bakes in the buffers' addresses: keep this object (and
+    the layer's weights and workspace) alive while replaying."""
+
+    def __init__(self, layer: MoELayer, x, noise=None):
+        self.layer = layer
+        self.x = x
+        self.noise = noise
+        self.y = torch.empty_like(x)
+        layer._reserve(x.shape[0], x.dtype)
+        side = torch.cuda.Stream(device=x.device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer(x, noise=noise, y=self.y)   # first call outside the capture
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize(x.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            layer(x, noise=noise, y=self.y)
+
+    def replay(self):
+        self.graph.replay()
+        return self.y

@@ -162,3 +162,25 @@ def test_status_clean_after_forward():
     layer(case.x, noise=case.noise)
     code, word = moe.check_status(layer.workspace)
     assert code == 0 and word == 0
+
+
+def test_graph_replay_matches_eager_and_follows_new_inputs():
+    """The forward captured in a CUDA graph gives the eager result bit for bit,
+    and replays on whatever was copied into its static input buffer."""
+    for name in ("decode_small", "mixtral_small"):
+        wl = SMALL[name]
+        case = Case(wl, seed=4)
+        layer = moe.MoELayer(case.W_g, case.W_up, case.W_down, wl.k, wl.cf, b_g=case.b_g, sigma=wl.sigma)
+        x0 = case.x.clone()
+        g = moe.GraphedForward(layer, x0, None if case.noise is None else case.noise.clone())
+        y_eager = layer(case.x, noise=case.noise)
+        torch.cuda.synchronize()
+        assert torch.equal(g.replay().view(torch.int16), y_eager.view(torch.int16))
+        other = Case(wl, seed=9)
+        g.x.copy_(other.x)
+        if g.noise is not None:
+            g.noise.copy_(other.noise)
+        y_new = g.replay().clone()
+        y_ref = layer(other.x, noise=other.noise)
+        torch.cuda.synchronize()
+        assert torch.equal(y_new.view(torch.int16), y_ref.view(torch.int16))
