@@ -122,6 +122,30 @@ MOE_API moe_status moe_dispatch(const int32_t *topk_idx, const void *x, moe_dtyp
                         int32_t *offsets, void *x_gathered, void *ws, size_t ws_bytes,
                         void *stream);
 
+/* Dispatch without a caller workspace.  No counterpart in the pages: this is
+ * for callers that cannot allocate device memory when they dispatch, such as a
+ * host runtime that forbids cudaMalloc after start-up (a device allocation can
+ * synchronise the GPU and stall the latency-critical path) or a plug-in whose
+ * framework owns every byte of device memory and hands it no scratch.
+ *
+ * Same arguments, results and errors as moe_dispatch, minus ws/ws_bytes.  The
+ * scratch (per-block histograms and totals) lives in one fixed 8 MiB device
+ * array inside the library, which every GPU that loads the library holds until
+ * the process exits; batches needing more (moe_dispatch_workspace_size() >
+ * 8 MiB, i.e. about N * k * E > 2^29) get MOE_ERR_INVALID_ARG with a
+ * message.  The call allocates nothing and calls no allocating routine.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) for that device; make that first call before any
+ *    stream capture on the device.
+ *  - Every call shares the one array and leaves its contents behind; the
+ *    passes overwrite every scratch entry they read, so nothing has to start
+ *    at zero.
+ *  - Calls whose kernels overlap on the GPU (other streams, other threads)
+ *    race on the array: serialise them. */
+MOE_API moe_status moe_dispatch_noalloc(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N,
+                                        int d, int E, int k, double cf, int32_t *slot, int32_t *counts,
+                                        int32_t *offsets, void *x_gathered, void *stream);
+
 /* ---------------------------------------------------------------- experts */
 
 /* Workspace bytes for moe_expert_ffn (status word + the hidden activations). */

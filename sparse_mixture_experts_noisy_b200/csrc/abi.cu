@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "../../include/moe.h"
@@ -133,6 +134,34 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
     return MOE_OK;
 }
 
+// ---------------------------------------------------------------- dispatch without a workspace
+// Scratch for moe_dispatch_noalloc: the per-block histograms and the
+// per-(choice, expert) totals of the dispatch passes, in a fixed device array
+// that every GPU loading this library holds until the process exits.
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t noalloc_scratch_address(void **out) {
+    static std::mutex mu;
+    static void *addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -205,6 +234,36 @@ moe_status moe_dispatch(const int32_t *topk_idx, const void *x, moe_dtype dt, in
     REQUIRE_PTR(ws, "ws");
     cudaError_t e = moe::launch_dispatch(topk_idx, x, elem_bytes(dt), N, d, E, k, C, slot, counts,
                                          offsets, x_gathered, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
+    return MOE_OK;
+}
+
+moe_status moe_dispatch_noalloc(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N, int d,
+                                int E, int k, double cf, int32_t *slot, int32_t *counts,
+                                int32_t *offsets, void *x_gathered, void *stream) {
+    moe_status st = check_shape(N, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity factor must be > 0 or +inf (got %g)", cf);
+    REQUIRE_PTR(counts, "counts");
+    REQUIRE_PTR(offsets, "offsets");
+    if (N > 0) {
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(slot, "slot");
+        REQUIRE_PTR(x_gathered, "x_gathered");
+    }
+    const size_t need = moe::dispatch_ws_bytes(N, E, k);
+    if (need > kNoAllocScratchBytes)
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_dispatch_noalloc: N=%lld, E=%d, k=%d needs %zu bytes of scratch, more than its "
+                    "fixed %zu bytes; use moe_dispatch with a workspace",
+                    (long long)N, E, k, need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    cudaError_t e = noalloc_scratch_address(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_dispatch_noalloc scratch lookup");
+    e = moe::launch_dispatch(topk_idx, x, elem_bytes(dt), N, d, E, k, C, slot, counts, offsets, x_gathered,
+                             scratch, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dispatch launch");
     return MOE_OK;
 }

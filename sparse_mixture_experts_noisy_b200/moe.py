@@ -20,7 +20,7 @@ MOE_F32, MOE_BF16 = 0, 1
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
-EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch",
+EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
            "moe_forward", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
@@ -53,6 +53,7 @@ def load_library(path: str = LIB_PATH):
             "moe_route": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P]),
             "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
             "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
+            "moe_dispatch_noalloc": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P]),
             "moe_expert_ffn_workspace_size": (SZ, [I64, I, I, I, I]),
             "moe_expert_ffn": (I, [P, P, P, P, P, I, I64, I, I, I, P, P, SZ, P]),
             "moe_combine": (I, [P, P, P, P, P, I, I64, I, I, P, P]),
@@ -154,6 +155,31 @@ def moe_dispatch(topk_idx, x, E, cf, stream=None):
     ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
     _check(L.moe_dispatch(_p(topk_idx), _p(x), _dt(x), N, d, E, k, _cf(cf), _p(slot), _p(counts),
                           _p(offsets), _p(xg), _p(ws), ws.numel(), _stream(stream)))
+    return dict(slot=slot, counts=counts, offsets=offsets, x_gathered=xg, rows=rows,
+                C=capacity(N, E, k, cf))
+
+
+def moe_dispatch_noalloc(topk_idx, x, E, cf, stream=None):
+    """moe_dispatch for callers that cannot allocate device memory at dispatch
+    time: the library's fixed scratch array replaces the workspace.  The
+    output tensors here are allocated by torch for convenience; a caller
+    without an allocator passes its own buffers to the C entry point.
+    -> dict(slot, counts, offsets, x_gathered, rows, C)."""
+    L = load_library()
+    _cuda(topk_idx, "topk_idx")
+    _cuda(x, "x")
+    N, d = x.shape
+    k = topk_idx.shape[1]
+    dev = x.device
+    rows = L.moe_gathered_rows(N, E, k, _cf(cf))
+    if rows < 0:
+        raise MoeError(1, "invalid capacity arguments")
+    slot = torch.empty((N, k), dtype=torch.int32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    xg = torch.empty((rows, d), dtype=x.dtype, device=dev)
+    _check(L.moe_dispatch_noalloc(_p(topk_idx), _p(x), _dt(x), N, d, E, k, _cf(cf), _p(slot), _p(counts),
+                                  _p(offsets), _p(xg), _stream(stream)))
     return dict(slot=slot, counts=counts, offsets=offsets, x_gathered=xg, rows=rows,
                 C=capacity(N, E, k, cf))
 
