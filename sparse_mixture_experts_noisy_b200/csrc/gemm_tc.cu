@@ -34,6 +34,7 @@
 #include "internal.h"
 
 #include <cudaTypedefs.h>
+#include <cstdlib>
 
 namespace moe {
 
@@ -367,6 +368,258 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
     }
 }
 
+// ---------------------------------------------------------------- CTA-pair variant (prefill)
+// Two CTAs of a cluster share one 256 x 256 output tile (tcgen05 cta_group::2).
+// Each CTA loads, per 64-wide K block, its own 128 token rows of A and its own
+// 128 weight rows of B (plain TMA loads, no multicast) into a 6-stage ring; the
+// bytes of both CTAs complete on the leader's (rank 0) barrier.  The leader's
+// MMA lane issues M = 256, N = 256 MMAs that read A from each CTA's own shared
+// memory and B from both, accumulating each CTA's 128 rows in that CTA's tensor
+// memory; its commits arrive on both CTAs' barriers.  Both CTAs' epilogue warps
+// drain their own accumulators and report to the leader's barrier.  Per byte
+// moved from L2 this does a third more MMA work than the one-CTA tile, and each
+// stage is 32 KB, so the ring is 50 % deeper.
+template <int EPI, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
+                const TcArgs args) {
+    constexpr int BT = 256;                        // pair tile: 256 token rows x 256 weight rows
+    constexpr uint32_t A_BYTES = 128 * kBK * 2;    // this CTA's 128 token rows
+    constexpr uint32_t B_BYTES = 128 * kBK * 2;    // this CTA's 128 weight rows
+    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t TMEM_COLS = 512;            // two 256-column accumulators
+
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+    __shared__ uint32_t tmem_holder;
+    __shared__ int32_t pre_s[257];
+    __shared__ int32_t cnt_s[256];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int E = args.E, Nw = args.Nw, splits = args.splits;
+    const int kb_total = (args.K + kBK - 1) / kBK;
+    uint32_t *status = args.status;
+    const uint64_t tmo = args.timeout_ns;
+
+    const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    const uint32_t full0 = smem_u32(&bars[0]);
+    const uint32_t empty0 = smem_u32(&bars[STAGES]);
+    const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
+    const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+    const uint32_t full0_lead = map_to_cta(full0, 0);
+    const uint32_t tempty0_lead = map_to_cta(tempty0, 0);
+
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            pre_s[e] = run;
+            run += ((cnt_s[e] + BT - 1) / BT) * ((Nw + BT - 1) / BT) * splits;
+        }
+        pre_s[E] = run;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(tfull0, 1);
+        mbar_init(tfull0 + 8, 1);
+        mbar_init(tempty0, 8);       // 4 epilogue warps in each CTA
+        mbar_init(tempty0 + 8, 8);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_tok);
+        tma_prefetch_desc(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&tmem_holder), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before either signals the other
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_holder;
+    const int total_units = pre_s[E];
+
+    auto decode = [&](int u, int &e, int &tok0, int &w0, int &kb0, int &kb1, int &n_valid) {
+        int lo = 0, hi = E;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre_s[mid] <= u) lo = mid; else hi = mid;
+        }
+        e = lo;
+        int r = u - pre_s[lo];
+        const int split = r % splits;
+        r /= splits;
+        const int mt = (cnt_s[lo] + BT - 1) / BT;
+        tok0 = (r % mt) * BT;
+        w0 = (r / mt) * BT;
+        n_valid = min(BT, Nw - w0);
+        kb0 = static_cast<int>(static_cast<int64_t>(split) * kb_total / splits);
+        kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * kb_total / splits);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int issued = 0;
+            for (int u = pair; u < total_units && ok; u += npairs) {
+                int e, tok0, w0, kb0, kb1, nv;
+                decode(u, e, tok0, w0, kb0, kb1, nv);
+                const int tok_row = args.offsets[e] + tok0 + static_cast<int>(rank) * 128;
+                const int w_row = w0 + static_cast<int>(rank) * 128;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * STAGE_BYTES);
+                    const uint32_t fb = full0_lead + 8 * stage;
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const int kx = kb * kBK;
+                    tma_load_2d_pair(sa, &tm_tok, fb, kx, tok_row);
+                    tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, kx, w_row, e);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {
+                // the pair's copies of the stages armed here land before exit
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && i < issued; ++i) {
+                    if (st == 0) {
+                        st = STAGES - 1;
+                        ph ^= 1u;
+                    } else {
+                        --st;
+                    }
+                    wait_drain(full0 + 8 * st, ph, tmo);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, any = false;
+            int local = 0;
+            const uint32_t idesc = idesc_bf16_f32(256, 256);
+            for (int u = pair; u < total_units && ok; u += npairs) {
+                int e, tok0, w0, kb0, kb1, nv;
+                decode(u, e, tok0, w0, kb0, kb1, nv);
+                const int acc = local & 1;
+                const uint32_t acc_phase = (local >> 1) & 1;
+                if (!mbar_wait_bounded(tempty0 + 8 * acc, acc_phase ^ 1u, status, tmo, 12)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BT);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(full0 + 8 * stage, phase, status, tmo, 13)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint64_t ad = smem_desc_sw128(sa);
+                    const uint64_t bd = smem_desc_sw128(sa + A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                    any = true;
+                    umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair_mc(tfull0 + 8 * acc, 0x3);
+                ++local;
+            }
+            if (!ok && any) {
+                umma_commit_pair(drain);
+                wait_drain(drain, 0, tmo);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int u = pair; u < total_units; u += npairs) {
+            int e, tok0, w0, kb0, kb1, nv;
+            decode(u, e, tok0, w0, kb0, kb1, nv);
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            const bool mine = mbar_wait_bounded(tfull0 + 8 * acc, acc_phase, status, tmo, 14);
+            if (!__all_sync(0xffffffffu, mine)) break;
+            tc_fence_after();
+            const int cnt = cnt_s[e];
+            const int my_row = tok0 + static_cast<int>(rank) * 128 + row_in_tile;
+            const bool rv = my_row < cnt;
+            const int64_t grow = static_cast<int64_t>(args.offsets[e]) + my_row;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * BT);
+            const int chunks = (nv + 31) >> 5;
+            for (int c = 0; c < chunks; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_wait_ld();
+                if (EPI == EPI_BF16_RELU) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
+                }
+                const int col0 = w0 + c * 32;
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int col = col0 + 8 * g;
+                    if (rv && col < Nw) {
+                        uint4 v;
+                        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            h[i] = __floats2bfloat162_rn(__uint_as_float(r[8 * g + 2 * i]),
+                                                         __uint_as_float(r[8 * g + 2 * i + 1]));
+                        *reinterpret_cast<uint4 *>(o + col) = v;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(tempty0 + 8 * acc);
+                else mbar_arrive_cluster(tempty0_lead + 8 * acc);
+            }
+            ++local;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    cluster_sync();  // the pair's MMAs and remote arrivals are done before TMEM goes
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -428,6 +681,33 @@ cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, i
     return cudaGetLastError();
 }
 
+template <int EPI, int STAGES>
+cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
+                       const int32_t *offsets, const int32_t *counts, void *out, int64_t ldo,
+                       uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s) {
+    CUtensorMap tm_tok, tm_w;
+    if (!make_map_2d(&tm_tok, tok, tok_rows, K, 128)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
+    constexpr int smem = STAGES * 2 * 128 * kBK * 2 + 1024;
+    auto kern = tc2_gemm_kernel<EPI, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int pairs = num_sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    int max_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) == cudaSuccess && max_clusters > 0 &&
+        max_clusters < pairs)
+        pairs = max_clusters;
+    (void)cudaGetLastError();
+    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns};
+    kern<<<2 * pairs, kThreads, smem, s>>>(tm_tok, tm_w, a);
+    return cudaGetLastError();
+}
+
 // Sum of K-split fp32 partials into dtype rows, in split order.
 __global__ void __launch_bounds__(256)
 reduce_parts_kernel(const float *__restrict__ parts, int nparts, int64_t part_stride,
@@ -454,6 +734,12 @@ TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
     TcPlan p{};
     p.decode = rows <= 256;
     p.splits_down = 1;
+    // CTA-pair tiles for prefill; MOE_TC_PAIR=0 selects the one-CTA tiles
+    static const int pair_env = [] {
+        const char *v = getenv("MOE_TC_PAIR");
+        return v ? atoi(v) : 1;
+    }();
+    p.pair = !p.decode && pair_env != 0 && num_sms >= 2;
     if (p.decode) {
         const int64_t units = static_cast<int64_t>(E) * ((d + kBM - 1) / kBM);
         const int kb_total = (d_ff + kBK - 1) / kBK;
@@ -481,6 +767,13 @@ cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t 
     const TcPlan p = plan_tc_ffn(rows, d, d_ff, E, num_sms);
     if (plan_out) *plan_out = p;
     cudaError_t e;
+    if (!p.decode && p.pair) {
+        e = launch_tc2<EPI_BF16_RELU, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
+                                         timeout_ns, num_sms, s);
+        if (e != cudaSuccess) return e;
+        return launch_tc2<EPI_BF16, 6>(H, rows, W_down, E, d, d_ff, offsets, counts, out, d, status,
+                                       timeout_ns, num_sms, s);
+    }
     if (!p.decode) {
         e = launch_tc<256, false, EPI_BF16_RELU, 4>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H,
                                                     d_ff, 0, status, timeout_ns, num_sms, s);

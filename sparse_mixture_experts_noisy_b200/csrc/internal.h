@@ -42,6 +42,7 @@ cudaError_t launch_simt_ffn(const void *xg, const int32_t *offsets, const int32_
 // Tensor-core expert FFN (gemm_tc.cu).
 struct TcPlan {
     bool decode;      // weight rows as the MMA's M (few tokens per expert)
+    bool pair;        // prefill on CTA pairs (tcgen05 cta_group::2)
     int splits_down;  // K splits of the down projection (decode only)
 };
 TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms);
