@@ -391,7 +391,7 @@ def roofline_entry(kind, achieved, peak, unit, traffic, kernel, peak_src, extra=
 def run_ours(args):
     import torch
     from sparse_mixture_experts_noisy_b200 import moe
-    from sparse_mixture_experts_noisy_b200.synth import WORKLOADS, make_inputs
+    from sparse_mixture_experts_noisy_b200.synth import WORKLOADS, make_inputs, make_noise, make_x
 
     dist = Dist("nccl")
     torch.cuda.set_device(dist.local_rank)
@@ -399,7 +399,11 @@ def run_ours(args):
     moe.load_library()
     peaks, peak_src = load_peaks()
     wl = WORKLOADS[args.workload]
-    inp = make_inputs(wl, args.seed + dist.rank)
+    # replicas of one model: the same weights on every rank, each rank its own tokens
+    inp = make_inputs(wl, args.seed)
+    if dist.rank > 0:
+        inp.x = make_x(wl, args.seed + 7919 * dist.rank)
+        inp.noise = make_noise(wl, args.seed + 7919 * dist.rank)
     inp_dev = tuple(to_dev(a, torch) for a in (inp.x, inp.W_g, inp.b_g, inp.noise, inp.W_up, inp.W_down))
     weights_bytes = 2 * wl.E * wl.d * wl.d_ff * (2 if wl.dtype == "bf16" else 4)
     flush = weights_bytes <= L2_BYTES
@@ -415,12 +419,17 @@ def run_ours(args):
     elem = 2 if wl.dtype == "bf16" else 4
     tc = wl.dtype == "bf16" and wl.d % 8 == 0 and wl.d_ff % 8 == 0
     decode_plan = tc and moe.gathered_rows(wl.N, wl.E, wl.k, wl.cf) <= 256
-    kernel = "tc_gemm_kernel (up + down launches of one moe_expert_ffn call)" if tc else \
-             "simt_gemm_kernel (up + down)"
+    if not tc:
+        kernel = "simt_gemm_kernel (up + down)"
+    elif os.environ.get("MOE_TC_PAIR", "1") != "0":
+        kernel = "tc2_gemm_kernel, CTA pairs (up + down launches of one moe_expert_ffn call)"
+    else:
+        kernel = "tc_gemm_kernel (up + down launches of one moe_expert_ffn call)"
     if decode_plan:
         byt = ffn_bytes(counts, wl.d, wl.d_ff, elem)
         roof = roofline_entry("hbm", byt / ffn_sec / 1e9, peaks["hbm_gbs"], "GB/s",
-                              ncu_traffic("decode"), kernel + " + reduce_parts_kernel", peak_src + " (copy)",
+                              ncu_traffic("decode"), "tc_gemm_kernel, weight-row tiles (up + down) + reduce_parts_kernel",
+                              peak_src + " (copy)",
                               {"algorithmic_bytes": byt, "ms_per_call": ffn_sec * 1e3})
     else:
         fl = ffn_flops(R, wl.d, wl.d_ff)
@@ -451,7 +460,7 @@ def run_ours(args):
     # Mixtral-shaped one; measure it too when running that workload
     if args.workload == "mixtral" and not args.no_decode:
         dwl = WORKLOADS["decode"]
-        dinp = make_inputs(dwl, args.seed + dist.rank, weights=False)
+        dinp = make_inputs(dwl, args.seed + 7919 * dist.rank, weights=False)
         ddev = (to_dev(dinp.x, torch), inp_dev[1], None, None, inp_dev[4], inp_dev[5])
         dsteps = max(20, args.steps)
         dlayer, _, dsec, dclk = measure_layer(dwl, ddev, dsteps, args.warmup, dist, torch, moe, False)

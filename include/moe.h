@@ -57,6 +57,10 @@ extern "C" {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
+/* Expert activation: ReLU (the walkthrough's STEP 9) or GELU, x * Phi(x) with
+ * Phi the standard normal CDF (nanoMoE's MLPExperts, "nanoMoEの深層解剖" slide 32). */
+typedef enum { MOE_ACT_RELU = 1, MOE_ACT_GELU = 2 } moe_activation;
+
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,   /* bad size, null required pointer, misaligned pointer */
@@ -146,6 +150,46 @@ MOE_API moe_status moe_dispatch_noalloc(const int32_t *topk_idx, const void *x, 
                                         int d, int E, int k, double cf, int32_t *slot, int32_t *counts,
                                         int32_t *offsets, void *x_gathered, void *stream);
 
+/* ---------------------------------------------------------------- token-sharded batches */
+
+/* One batch whose tokens are split over G GPUs in contiguous ranges, rank
+ * order.  A queue place depends on every earlier token of the batch (all first
+ * choices before all second choices, "nanoMoEの深層解剖" slides 17-20), so the
+ * shards exchange their per-(choice, expert) counts once; everything else stays
+ * on each GPU.  Per shard:
+ *   moe_route                       (local tokens)
+ *   moe_shard_count   -> counts_je  (this shard's [k][E] totals)
+ *   all-gather counts_je over the G ranks (e.g. NCCL) into all_counts [G][k][E]
+ *   moe_shard_base    -> base       (this shard's first place per (j, e))
+ *   moe_shard_dispatch              (C = moe_capacity(N of the whole batch, ...))
+ *   moe_expert_ffn, moe_combine     (unchanged, on the shard's rows)
+ * The drop set equals the unsharded one; the combine output of every token is
+ * the same as in an unsharded call.  `slot` here numbers each expert's kept
+ * rows inside the shard (choice rank first, then token order).
+ *
+ * Workspace for the count/dispatch pair of one shard (the count pass leaves
+ * per-block prefixes in it that the dispatch reads: give both calls the same
+ * workspace and do not touch it in between). */
+MOE_API size_t moe_shard_workspace_size(int64_t N_local, int E, int k);
+
+/*  counts_je device [k][E] int32 out: this shard's number of j-th choices of e. */
+MOE_API moe_status moe_shard_count(const int32_t *topk_idx, int64_t N_local, int E, int k, int32_t *counts_je,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*  all_counts device [G][k][E] int32 (rank order); base device [k][E] int32 out:
+ *  base[j][e] = sum over all shards of choices j' < j of e + sum over shards
+ *  before `rank` of choice j of e. */
+MOE_API moe_status moe_shard_base(const int32_t *all_counts, int G, int rank, int E, int k, int32_t *base,
+                                  void *stream);
+
+/*  As moe_dispatch for this shard's tokens, with C the whole batch's capacity,
+ *  counts_je/ws from moe_shard_count and base from moe_shard_base.  x_gathered
+ *  needs ceil(N_local * k / 128) * 128 rows. */
+MOE_API moe_status moe_shard_dispatch(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N_local,
+                                      int d, int E, int k, int64_t C, const int32_t *counts_je,
+                                      const int32_t *base, int32_t *slot, int32_t *counts, int32_t *offsets,
+                                      void *x_gathered, void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- experts */
 
 /* Workspace bytes for moe_expert_ffn (status word + the hidden activations). */
@@ -169,6 +213,17 @@ MOE_API moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets
                           const void *W_up, const void *W_down, moe_dtype dt, int64_t rows,
                           int d, int d_ff, int E, void *out_gathered, void *ws, size_t ws_bytes,
                           void *stream);
+
+/* The nanoMoE expert variant ("nanoMoEの深層解剖" slide 32, MLPExperts):
+ *   out[r] = W_down[e] act(W_up[e] x_gathered[r] + b_up[e]) + b_down[e]
+ * activation: MOE_ACT_RELU or MOE_ACT_GELU (erf form); b_up device [E, d_ff]
+ * fp32 and b_down device [E, d] fp32, each nullable.  Everything else as
+ * moe_expert_ffn (which is this call with ReLU and no biases).  Dropout, which
+ * the slides apply in training, is the identity in this forward pass. */
+MOE_API moe_status moe_expert_ffn_ex(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                                     const void *W_up, const void *W_down, moe_dtype dt, int64_t rows, int d,
+                                     int d_ff, int E, int activation, const float *b_up, const float *b_down,
+                                     void *out_gathered, void *ws, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------- combine */
 
@@ -198,6 +253,17 @@ MOE_API moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, co
                        float *logits_out, int32_t *topk_out, float *gates_out,
                        int32_t *slot_out, int32_t *counts_out,
                        void *ws, size_t ws_bytes, void *stream);
+
+/* moe_forward with the nanoMoE expert variant (see moe_expert_ffn_ex):
+ * activation, b_up [E, d_ff] and b_down [E, d] (fp32, nullable).  moe_forward is
+ * this call with MOE_ACT_RELU and no biases.  Same workspace size. */
+MOE_API moe_status moe_forward_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                                  const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
+                                  int k, double cf, const void *W_up, const void *W_down, int activation,
+                                  const float *b_up, const float *b_down, void *y,
+                                  float *logits_out, int32_t *topk_out, float *gates_out,
+                                  int32_t *slot_out, int32_t *counts_out,
+                                  void *ws, size_t ws_bytes, void *stream);
 
 /* Number of kernels one moe_forward call with these arguments launches on its
  * stream (0 for N = 0, -1 for invalid arguments).  Useful to size CUDA-graph

@@ -153,29 +153,50 @@ void oracle_assign_slots(const int32_t *topk_idx, int64_t N, int E, int k, int64
     free(queue);
 }
 
-/* STEP 8-10 for one token and one expert, in double:
- *   z = W_up[e] x,  h = max(0, z),  o = W_down[e] h. */
-void oracle_expert_ffn(const void *x, int dt, const void *W_up, const void *W_down,
-                       int64_t t, int e, int d, int d_ff, double *h, double *o)
+/* The nanoMoE expert variant ("nanoMoEの深層解剖" slide 32, MLPExperts): an
+ * optional bias after each projection and GELU in place of ReLU.  GELU is the
+ * exact form x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), in double.
+ *   z = W_up[e] x + b_up[e],  h = act(z),  o = W_down[e] h + b_down[e]
+ * act: 1 = ReLU, 2 = GELU.  b_up [E][d_ff] and b_down [E][d] are fp32 or NULL. */
+void oracle_expert_ffn_ex(const void *x, int dt, const void *W_up, const void *W_down,
+                          const float *b_up, const float *b_down, int act,
+                          int64_t t, int e, int d, int d_ff, double *h, double *o)
 {
     for (int f = 0; f < d_ff; ++f) {
         double z = 0.0;
         size_t wrow = ((size_t)e * d_ff + f) * d;
         for (int i = 0; i < d; ++i)
             z += elem(W_up, dt, wrow + i) * elem(x, dt, (size_t)t * d + i);
-        h[f] = z > 0.0 ? z : 0.0;
+        if (b_up)
+            z += (double)b_up[(size_t)e * d_ff + f];
+        if (act == 2)
+            h[f] = 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
+        else
+            h[f] = z > 0.0 ? z : 0.0;
     }
     for (int i = 0; i < d; ++i) {
         double acc = 0.0;
         size_t wrow = ((size_t)e * d + i) * d_ff;
         for (int f = 0; f < d_ff; ++f)
             acc += elem(W_down, dt, wrow + f) * h[f];
+        if (b_down)
+            acc += (double)b_down[(size_t)e * d + i];
         o[i] = acc;
     }
 }
 
+/* STEP 8-10 for one token and one expert, in double:
+ *   z = W_up[e] x,  h = max(0, z),  o = W_down[e] h. */
+void oracle_expert_ffn(const void *x, int dt, const void *W_up, const void *W_down,
+                       int64_t t, int e, int d, int d_ff, double *h, double *o)
+{
+    oracle_expert_ffn_ex(x, dt, W_up, W_down, NULL, NULL, 1, t, e, d, d_ff, h, o);
+}
+
 struct combine_job {
     const void *x, *W_up, *W_down;
+    const float *b_up, *b_down;
+    int act;
     int dt;
     const int32_t *topk_idx, *slot;
     const float *gates;
@@ -203,7 +224,8 @@ static void *combine_range(void *arg)
                 continue;
             int e = jb->topk_idx[(size_t)t * jb->k + j];
             double g = (double)jb->gates[(size_t)t * jb->k + j];
-            oracle_expert_ffn(jb->x, jb->dt, jb->W_up, jb->W_down, t, e, jb->d, jb->d_ff, h, o);
+            oracle_expert_ffn_ex(jb->x, jb->dt, jb->W_up, jb->W_down, jb->b_up, jb->b_down, jb->act, t, e,
+                                 jb->d, jb->d_ff, h, o);
             for (int i = 0; i < jb->d; ++i)
                 yt[i] += g * o[i];
         }
@@ -213,13 +235,15 @@ static void *combine_range(void *arg)
     return NULL;
 }
 
-/* Layer output for the listed tokens (y rows in list order, double).
+/* Layer output for the listed tokens (y rows in list order, double), with the
+ * expert variant of oracle_expert_ffn_ex (act 1 = ReLU, 2 = GELU; biases nullable).
  * Work is split over tokens across nthreads plain threads; each token's
  * arithmetic is the same as with one thread. */
-void oracle_ffn_combine(const void *x, int dt, const void *W_up, const void *W_down,
-                        const int32_t *topk_idx, const float *gates, const int32_t *slot,
-                        int d, int d_ff, int k, const int64_t *tokens, int64_t n_tokens,
-                        double *y, int nthreads)
+void oracle_ffn_combine_ex(const void *x, int dt, const void *W_up, const void *W_down,
+                           const float *b_up, const float *b_down, int act,
+                           const int32_t *topk_idx, const float *gates, const int32_t *slot,
+                           int d, int d_ff, int k, const int64_t *tokens, int64_t n_tokens,
+                           double *y, int nthreads)
 {
     if (nthreads < 1)
         nthreads = 1;
@@ -230,6 +254,7 @@ void oracle_ffn_combine(const void *x, int dt, const void *W_up, const void *W_d
     for (int w = 0; w < nthreads; ++w) {
         struct combine_job *jb = &jobs[w];
         jb->x = x; jb->W_up = W_up; jb->W_down = W_down; jb->dt = dt;
+        jb->b_up = b_up; jb->b_down = b_down; jb->act = act;
         jb->topk_idx = topk_idx; jb->slot = slot; jb->gates = gates;
         jb->d = d; jb->d_ff = d_ff; jb->k = k; jb->tokens = tokens; jb->y = y;
         jb->begin = n_tokens * w / nthreads;
@@ -245,4 +270,14 @@ void oracle_ffn_combine(const void *x, int dt, const void *W_up, const void *W_d
     }
     free(jobs);
     free(th);
+}
+
+/* The layer as the walkthrough defines it: ReLU experts, no biases. */
+void oracle_ffn_combine(const void *x, int dt, const void *W_up, const void *W_down,
+                        const int32_t *topk_idx, const float *gates, const int32_t *slot,
+                        int d, int d_ff, int k, const int64_t *tokens, int64_t n_tokens,
+                        double *y, int nthreads)
+{
+    oracle_ffn_combine_ex(x, dt, W_up, W_down, NULL, NULL, 1, topk_idx, gates, slot, d, d_ff, k,
+                          tokens, n_tokens, y, nthreads);
 }

@@ -54,6 +54,10 @@ def _load():
             lib.oracle_expert_ffn.restype = None
             lib.oracle_ffn_combine.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, P, I64, P, I32]
             lib.oracle_ffn_combine.restype = None
+            lib.oracle_expert_ffn_ex.argtypes = [P, I32, P, P, P, P, I32, I64, I32, I32, I32, P, P]
+            lib.oracle_expert_ffn_ex.restype = None
+            lib.oracle_ffn_combine_ex.argtypes = [P, I32, P, P, P, P, I32, P, P, P, I32, I32, I32, P, I64, P, I32]
+            lib.oracle_ffn_combine_ex.restype = None
             _lib = lib
     return _lib
 
@@ -123,7 +127,27 @@ def expert_ffn(x, W_up, W_down, t, e):
     return h, o
 
 
-def ffn_combine(x, W_up, W_down, topk_idx, gates, slot, tokens=None, nthreads=1):
+ACT_RELU, ACT_GELU = 1, 2
+
+
+def expert_ffn_ex(x, W_up, W_down, t, e, act=ACT_RELU, b_up=None, b_down=None):
+    """(h, o) for the nanoMoE expert variant (slide 32): optional biases, ReLU or GELU."""
+    x = np.ascontiguousarray(x)
+    W_up = np.ascontiguousarray(W_up)
+    W_down = np.ascontiguousarray(W_down)
+    _, d = x.shape
+    d_ff = W_up.shape[1]
+    h = np.empty(d_ff, dtype=np.float64)
+    o = np.empty(d, dtype=np.float64)
+    bu = None if b_up is None else np.ascontiguousarray(b_up, dtype=np.float32)
+    bd = None if b_down is None else np.ascontiguousarray(b_down, dtype=np.float32)
+    _load().oracle_expert_ffn_ex(_ptr(x), _dt(x), _ptr(W_up), _ptr(W_down), _ptr(bu), _ptr(bd), int(act),
+                                 int(t), int(e), d, d_ff, _ptr(h), _ptr(o))
+    return h, o
+
+
+def ffn_combine(x, W_up, W_down, topk_idx, gates, slot, tokens=None, nthreads=1, act=ACT_RELU,
+                b_up=None, b_down=None):
     """y rows (float64) for the listed tokens (STEP 11-12; slides 38-40)."""
     x = np.ascontiguousarray(x)
     W_up = np.ascontiguousarray(W_up)
@@ -138,14 +162,16 @@ def ffn_combine(x, W_up, W_down, topk_idx, gates, slot, tokens=None, nthreads=1)
         tokens = np.arange(N, dtype=np.int64)
     tokens = np.ascontiguousarray(tokens, dtype=np.int64)
     y = np.empty((len(tokens), d), dtype=np.float64)
-    _load().oracle_ffn_combine(_ptr(x), _dt(x), _ptr(W_up), _ptr(W_down), _ptr(topk_idx),
-                               _ptr(gates), _ptr(slot), d, d_ff, k, _ptr(tokens), len(tokens),
-                               _ptr(y), int(nthreads))
+    bu = None if b_up is None else np.ascontiguousarray(b_up, dtype=np.float32)
+    bd = None if b_down is None else np.ascontiguousarray(b_down, dtype=np.float32)
+    _load().oracle_ffn_combine_ex(_ptr(x), _dt(x), _ptr(W_up), _ptr(W_down), _ptr(bu), _ptr(bd), int(act),
+                                  _ptr(topk_idx), _ptr(gates), _ptr(slot), d, d_ff, k, _ptr(tokens),
+                                  len(tokens), _ptr(y), int(nthreads))
     return y
 
 
 def forward(x, W_g, b_g, noise, sigma, k, cf, W_up, W_down, logits=None, tokens=None,
-            nthreads=1):
+            nthreads=1, act=ACT_RELU, b_up=None, b_down=None):
     """The whole layer.  ``logits`` (optional) replaces the oracle's own s_raw,
     so routing can be replayed from another implementation's fp32 logits.
     Returns a dict with every intermediate."""
@@ -155,6 +181,6 @@ def forward(x, W_g, b_g, noise, sigma, k, cf, W_up, W_down, logits=None, tokens=
     topk_idx, gates = route_from_logits(s_raw, k, noise, sigma)
     C = capacity(N, E, k, cf)
     slot, counts = assign_slots(topk_idx, E, C)
-    y = ffn_combine(x, W_up, W_down, topk_idx, gates, slot, tokens, nthreads)
+    y = ffn_combine(x, W_up, W_down, topk_idx, gates, slot, tokens, nthreads, act, b_up, b_down)
     return dict(s_raw=s_raw, topk_idx=topk_idx, gates=gates, C=C, slot=slot, counts=counts,
                 y=y, tokens=tokens)

@@ -108,7 +108,7 @@ FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows,
 moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts, const void *W_up,
                    const void *W_down, moe_dtype dt, int64_t rows, int d, int d_ff, int E, void *out,
                    void *ffn_ws, bool combine_reads_parts, float **parts_out, int *nparts_out,
-                   uint32_t *status, cudaStream_t s) {
+                   uint32_t *status, cudaStream_t s, int act, const float *b_up, const float *b_down) {
     cudaError_t e;
     if (parts_out) *parts_out = nullptr;
     if (nparts_out) *nparts_out = 0;
@@ -120,7 +120,7 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
         float *parts = p.decode ? reinterpret_cast<float *>(w + moe::align_up(static_cast<size_t>(rows) * d_ff * 2, 256))
                                 : nullptr;
         e = moe::launch_tc_ffn(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E, out, H, parts,
-                               combine_reads_parts, status, kWaitTimeoutNs, sms, s, nullptr);
+                               combine_reads_parts, status, kWaitTimeoutNs, sms, s, nullptr, act, b_up, b_down);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core expert FFN launch");
         if (p.decode && combine_reads_parts) {
             if (parts_out) *parts_out = parts;
@@ -129,7 +129,7 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
         return MOE_OK;
     }
     e = moe::launch_simt_ffn(xg, offsets, counts, W_up, W_down, dt == MOE_BF16 ? 1 : 0, rows, d, d_ff,
-                             E, out, ffn_ws, s);
+                             E, out, ffn_ws, s, act, b_up, b_down);
     if (e != cudaSuccess) return cuda_fail(e, "CUDA-core expert FFN launch");
     return MOE_OK;
 }
@@ -268,16 +268,79 @@ moe_status moe_dispatch_noalloc(const int32_t *topk_idx, const void *x, moe_dtyp
     return MOE_OK;
 }
 
+size_t moe_shard_workspace_size(int64_t N_local, int E, int k) {
+    if (N_local < 0 || E < 1 || k < 1) return 0;
+    return moe::dispatch_ws_bytes(N_local, E, k);
+}
+
+moe_status moe_shard_count(const int32_t *topk_idx, int64_t N_local, int E, int k, int32_t *counts_je,
+                           void *ws, size_t ws_bytes, void *stream) {
+    moe_status st = check_shape(N_local, 1, E, k, MOE_BF16);
+    if (st != MOE_OK) return st;
+    REQUIRE_PTR(counts_je, "counts_je");
+    if (N_local > 0) REQUIRE_PTR(topk_idx, "topk_idx");
+    const size_t need = moe::dispatch_ws_bytes(N_local, E, k);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "shard workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaError_t e = moe::launch_shard_count(topk_idx, N_local, E, k, counts_je, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard count launch");
+    return MOE_OK;
+}
+
+moe_status moe_shard_base(const int32_t *all_counts, int G, int rank, int E, int k, int32_t *base,
+                          void *stream) {
+    if (G < 1 || rank < 0 || rank >= G) return fail(MOE_ERR_INVALID_ARG, "need 0 <= rank < G (got rank=%d, G=%d)", rank, G);
+    if (E < 1 || E > 256 || k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "bad E or k");
+    REQUIRE_PTR(all_counts, "all_counts");
+    REQUIRE_PTR(base, "base");
+    cudaError_t e = moe::launch_shard_base(all_counts, G, rank, E, k, base, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard base launch");
+    return MOE_OK;
+}
+
+moe_status moe_shard_dispatch(const int32_t *topk_idx, const void *x, moe_dtype dt, int64_t N_local, int d,
+                              int E, int k, int64_t C, const int32_t *counts_je, const int32_t *base,
+                              int32_t *slot, int32_t *counts, int32_t *offsets, void *x_gathered, void *ws,
+                              size_t ws_bytes, void *stream) {
+    moe_status st = check_shape(N_local, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity must be >= 0 (got %lld)", (long long)C);
+    REQUIRE_PTR(counts, "counts");
+    REQUIRE_PTR(offsets, "offsets");
+    if (N_local > 0) {
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(counts_je, "counts_je");
+        REQUIRE_PTR(base, "base");
+        REQUIRE_PTR(slot, "slot");
+        REQUIRE_PTR(x_gathered, "x_gathered");
+    }
+    const size_t need = moe::dispatch_ws_bytes(N_local, E, k);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "shard workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaError_t e = moe::launch_shard_dispatch(topk_idx, x, elem_bytes(dt), N_local, d, E, k, C, counts_je, base,
+                                               slot, counts, offsets, x_gathered, ws,
+                                               static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "shard dispatch launch");
+    return MOE_OK;
+}
+
 size_t moe_expert_ffn_workspace_size(int64_t rows, int d, int E, int d_ff, moe_dtype dt) {
     if (rows < 0 || d < 1 || E < 1 || d_ff < 1 || (dt != MOE_F32 && dt != MOE_BF16)) return 0;
     return moe::kStatusBytes + ffn_ws_bytes(rows, d, E, d_ff, dt);
 }
 
-moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
-                          const void *W_up, const void *W_down, moe_dtype dt, int64_t rows,
-                          int d, int d_ff, int E, void *out_gathered, void *ws, size_t ws_bytes,
-                          void *stream) {
+moe_status moe_expert_ffn_ex(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                             const void *W_up, const void *W_down, moe_dtype dt, int64_t rows, int d,
+                             int d_ff, int E, int activation, const float *b_up, const float *b_down,
+                             void *out_gathered, void *ws, size_t ws_bytes, void *stream) {
     if (dt != MOE_F32 && dt != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+    if (activation != MOE_ACT_RELU && activation != MOE_ACT_GELU)
+        return fail(MOE_ERR_INVALID_ARG, "activation must be MOE_ACT_RELU or MOE_ACT_GELU");
     if (rows < 0 || rows % 128 != 0)
         return fail(MOE_ERR_INVALID_ARG, "rows must be a non-negative multiple of 128 (moe_gathered_rows)");
     if (d < 1 || d_ff < 1 || E < 1 || E > 256) return fail(MOE_ERR_INVALID_ARG, "bad d, d_ff or E");
@@ -286,6 +349,8 @@ moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const 
     REQUIRE_PTR(counts, "counts");
     REQUIRE_PTR(W_up, "W_up");
     REQUIRE_PTR(W_down, "W_down");
+    OPTIONAL_PTR(b_up, "b_up");
+    OPTIONAL_PTR(b_down, "b_down");
     if (rows > 0) {
         REQUIRE_PTR(x_gathered, "x_gathered");
         REQUIRE_PTR(out_gathered, "out_gathered");
@@ -301,7 +366,16 @@ moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const 
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     if (rows == 0) return MOE_OK;
     return run_ffn(x_gathered, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, out_gathered,
-                   static_cast<uint8_t *>(ws) + moe::kStatusBytes, false, nullptr, nullptr, status, s);
+                   static_cast<uint8_t *>(ws) + moe::kStatusBytes, false, nullptr, nullptr, status, s, activation,
+                   b_up, b_down);
+}
+
+moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                          const void *W_up, const void *W_down, moe_dtype dt, int64_t rows,
+                          int d, int d_ff, int E, void *out_gathered, void *ws, size_t ws_bytes,
+                          void *stream) {
+    return moe_expert_ffn_ex(x_gathered, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, MOE_ACT_RELU,
+                             nullptr, nullptr, out_gathered, ws, ws_bytes, stream);
 }
 
 moe_status moe_combine(const void *out_gathered, const int32_t *slot, const int32_t *topk_idx,
@@ -331,18 +405,23 @@ size_t moe_workspace_size(int64_t N, int d, int E, int d_ff, int k, double cf, m
     return forward_layout(N, d, E, d_ff, k, rows_for(N, E, k, C), dt).total;
 }
 
-moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
-                       const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
-                       int k, double cf, const void *W_up, const void *W_down, void *y,
-                       float *logits_out, int32_t *topk_out, float *gates_out,
-                       int32_t *slot_out, int32_t *counts_out,
-                       void *ws, size_t ws_bytes, void *stream) {
+moe_status moe_forward_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                          const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
+                          int k, double cf, const void *W_up, const void *W_down, int activation,
+                          const float *b_up, const float *b_down, void *y,
+                          float *logits_out, int32_t *topk_out, float *gates_out,
+                          int32_t *slot_out, int32_t *counts_out,
+                          void *ws, size_t ws_bytes, void *stream) {
     moe_status st = check_shape(N, d, E, k, dt);
     if (st != MOE_OK) return st;
     if (d_ff < 1) return fail(MOE_ERR_INVALID_ARG, "d_ff must be >= 1");
     const int64_t C = moe_capacity(N, E, k, cf);
     if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity factor must be > 0 or +inf (got %g)", cf);
     if (!std::isfinite(sigma)) return fail(MOE_ERR_INVALID_ARG, "sigma must be finite");
+    if (activation != MOE_ACT_RELU && activation != MOE_ACT_GELU)
+        return fail(MOE_ERR_INVALID_ARG, "activation must be MOE_ACT_RELU or MOE_ACT_GELU");
+    OPTIONAL_PTR(b_up, "b_up");
+    OPTIONAL_PTR(b_down, "b_down");
     REQUIRE_PTR(W_g, "W_g");
     REQUIRE_PTR(W_up, "W_up");
     REQUIRE_PTR(W_down, "W_down");
@@ -391,19 +470,35 @@ moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const floa
     float *parts = nullptr;
     int nparts = 0;
     st = run_ffn(xg, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, og, w + L.ffn, true, &parts,
-                 &nparts, status, s);
+                 &nparts, status, s, activation, b_up, b_down);
     if (st != MOE_OK) return st;
     e = moe::launch_combine(og, parts, nparts, rows * static_cast<int64_t>(d), slot, topk, offsets,
-                            gates, dt == MOE_BF16 ? 1 : 0, N, d, k, E, y, s);
+                            gates, dt == MOE_BF16 ? 1 : 0, N, d, k, E, y, s, nparts > 0 ? b_down : nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
     return MOE_OK;
+}
+
+moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                       const float *noise, float sigma, int64_t N, int d, int E, int d_ff,
+                       int k, double cf, const void *W_up, const void *W_down, void *y,
+                       float *logits_out, int32_t *topk_out, float *gates_out,
+                       int32_t *slot_out, int32_t *counts_out,
+                       void *ws, size_t ws_bytes, void *stream) {
+    return moe_forward_ex(x, dt, W_g, b_g, noise, sigma, N, d, E, d_ff, k, cf, W_up, W_down, MOE_ACT_RELU,
+                          nullptr, nullptr, y, logits_out, topk_out, gates_out, slot_out, counts_out, ws,
+                          ws_bytes, stream);
 }
 
 int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt) {
     if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1 || moe_capacity(N, E, k, cf) < 0) return -1;
     if (N == 0) return 0;
-    // router + dispatch passes + two expert GEMMs + combine
-    return 1 + moe::dispatch_launches(N, E, k) + 2 + 1;
+    int ffn = 2;
+    if (use_tensor_cores(dt, d, d_ff)) {
+        const int64_t rows = rows_for(N, E, k, moe_capacity(N, E, k, cf));
+        ffn = moe::tc_ffn_launches(moe::plan_tc_ffn(rows, d, d_ff, E, num_sms_current()), true);
+    }
+    // router + dispatch passes + expert FFN + combine
+    return 1 + moe::dispatch_launches(N, E, k) + ffn + 1;
 }
 
 moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {

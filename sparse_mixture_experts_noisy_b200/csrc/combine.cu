@@ -5,9 +5,9 @@
 // cb_weight @ exp_out: a dropped pair has weight 0, the kept ones keep their
 // gate, so a token whose choices were all dropped gets a zero row).
 // The dense [tokens, E*C] x [E*C, d] product of the slides is replaced by a
-// gather: a block takes one token at a time, each thread owns a chunk of its
-// output columns, reads that chunk of the token's k expert-output rows and
-// accumulates g * row in fp32, in choice order j = 0..k-1.
+// gather: for each token, threads own chunks of its output columns, read those
+// chunks of the token's k expert-output rows and accumulate g * row in fp32, in
+// choice order j = 0..k-1.  A block takes one token at a time.
 //
 // The expert outputs are either rows of dtype T (one partial) or `parts`
 // fp32 partial sums over K-splits of the down projection, which are added in
@@ -78,12 +78,15 @@ combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, 
                int64_t part_stride, const int32_t *__restrict__ slot,
                const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
                const float *__restrict__ gates, int64_t N, int d, int k, int E,
-               T *__restrict__ y) {
+               T *__restrict__ y, const float *__restrict__ b_down) {
+    pdl_trigger();
+    pdl_wait();
     // a block takes tokens in turn; its threads split the token's columns into
     // VEC-wide chunks; the token's k (row, gate) pairs are read once per block
     extern __shared__ int32_t c_smem[];
     int32_t *rows = c_smem;                                  // [k] source row or -1
     float *g = reinterpret_cast<float *>(rows + k);          // [k]
+    int32_t *re = rows + 2 * k;                              // [k] expert
     const int chunks = d / VEC;
     for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
         for (int j = threadIdx.x; j < k; j += blockDim.x) {
@@ -92,6 +95,7 @@ combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, 
             const bool ok = sl >= 0 && e >= 0 && e < E;
             rows[j] = ok ? offsets[e] + sl : -1;
             g[j] = ok ? gates[t * k + j] : 0.0f;
+            re[j] = ok ? e : 0;
         }
         __syncthreads();
         for (int ch = threadIdx.x; ch < chunks; ch += blockDim.x) {
@@ -107,11 +111,18 @@ combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, 
                     Vec<T, VEC>::load(out_rows + static_cast<int64_t>(r) * d + c, o);
                 } else {
                     load_f32<VEC>(parts + static_cast<int64_t>(r) * d + c, o);
+#pragma unroll 4
                     for (int p = 1; p < nparts; ++p) {
                         float q[VEC];
                         load_f32<VEC>(parts + p * part_stride + static_cast<int64_t>(r) * d + c, q);
 #pragma unroll
                         for (int v = 0; v < VEC; ++v) o[v] += q[v];
+                    }
+                    if (b_down != nullptr) {
+                        float bq[VEC];
+                        load_f32<VEC>(b_down + static_cast<int64_t>(re[j]) * d + c, bq);
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) o[v] += bq[v];
                     }
                 }
                 const float gj = g[j];
@@ -128,18 +139,17 @@ template <typename T, int VEC>
 cudaError_t launch_combine_t(const void *out_rows, const float *parts, int nparts,
                              int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
                              const int32_t *offsets, const float *gates, int64_t N, int d, int k,
-                             int E, void *y, cudaStream_t s) {
+                             int E, void *y, cudaStream_t s, const float *b_down) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int chunks = d / VEC;
     const int threads = chunks >= 256 ? 256 : (chunks >= 128 ? 128 : (chunks >= 64 ? 64 : 32));
     int64_t blocks = N;
     if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
-    const size_t smem = sizeof(int32_t) * 2 * static_cast<size_t>(k);
-    combine_kernel<T, VEC><<<static_cast<unsigned>(blocks), threads, smem, s>>>(
-        static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets, gates, N,
-        d, k, E, static_cast<T *>(y));
-    return cudaGetLastError();
+    const size_t smem = sizeof(int32_t) * 3 * static_cast<size_t>(k);
+    return launch_pdl(combine_kernel<T, VEC>, dim3(static_cast<unsigned>(blocks)), dim3(threads), smem, s,
+                      static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets, gates,
+                      N, d, k, E, static_cast<T *>(y), b_down);
 }
 
 }  // namespace
@@ -147,23 +157,24 @@ cudaError_t launch_combine_t(const void *out_rows, const float *parts, int npart
 cudaError_t launch_combine(const void *out_rows, const float *parts, int nparts,
                            int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
                            const int32_t *offsets, const float *gates, int dt, int64_t N, int d,
-                           int k, int E, void *y, cudaStream_t s) {
+                           int k, int E, void *y, cudaStream_t s, const float *b_down) {
     if (N == 0) return cudaSuccess;
     const bool al = (reinterpret_cast<uintptr_t>(y) % 16 == 0) &&
                     (reinterpret_cast<uintptr_t>(out_rows) % 16 == 0) &&
-                    (reinterpret_cast<uintptr_t>(parts) % 16 == 0);
+                    (reinterpret_cast<uintptr_t>(parts) % 16 == 0) &&
+                    (reinterpret_cast<uintptr_t>(b_down) % 16 == 0);
     if (dt == 1) {
         if (d % 8 == 0 && al)
             return launch_combine_t<__nv_bfloat16, 8>(out_rows, parts, nparts, part_stride, slot,
-                                                      topk_idx, offsets, gates, N, d, k, E, y, s);
+                                                      topk_idx, offsets, gates, N, d, k, E, y, s, b_down);
         return launch_combine_t<__nv_bfloat16, 1>(out_rows, parts, nparts, part_stride, slot,
-                                                  topk_idx, offsets, gates, N, d, k, E, y, s);
+                                                  topk_idx, offsets, gates, N, d, k, E, y, s, b_down);
     }
     if (d % 4 == 0 && al)
         return launch_combine_t<float, 4>(out_rows, parts, nparts, part_stride, slot, topk_idx,
-                                          offsets, gates, N, d, k, E, y, s);
+                                          offsets, gates, N, d, k, E, y, s, b_down);
     return launch_combine_t<float, 1>(out_rows, parts, nparts, part_stride, slot, topk_idx,
-                                      offsets, gates, N, d, k, E, y, s);
+                                      offsets, gates, N, d, k, E, y, s, b_down);
 }
 
 }  // namespace moe

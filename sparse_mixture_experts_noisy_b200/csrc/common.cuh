@@ -40,6 +40,13 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// Programmatic dependent launch: the next kernel on the stream may be scheduled
+// once every CTA of this grid has called pdl_trigger(); pdl_wait() blocks until
+// the previous kernel on the stream has finished and its writes are visible
+// (a no-op for a kernel launched without the attribute).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

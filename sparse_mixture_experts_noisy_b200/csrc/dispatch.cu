@@ -30,6 +30,8 @@ constexpr int kDispatchWarps = kDispatchTB / 32;
 __global__ void __launch_bounds__(kDispatchTB)
 hist_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k,
             int32_t *__restrict__ hist /* [nblk][k][E] */) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ int32_t h_smem[];  // [E]
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchTB + threadIdx.x;
     for (int j = 0; j < k; ++j) {
@@ -50,6 +52,8 @@ hist_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k,
 // place; the total goes to tot[j][e].
 __global__ void __launch_bounds__(256)
 scan_kernel(int32_t *__restrict__ hist, int nblk, int E, int k, int32_t *__restrict__ tot) {
+    pdl_trigger();
+    pdl_wait();
     const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (pair >= k * E) return;
@@ -77,6 +81,8 @@ assign_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int
               const int32_t *__restrict__ hist_excl /* [nblk][k][E] */,
               const int32_t *__restrict__ tot /* [k][E] */, int32_t *__restrict__ slot,
               int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ int32_t a_smem[];
     int32_t *warp_cnt = a_smem;                                // [warps][E]
     int32_t *jrun = warp_cnt + kDispatchWarps * E;             // [E]  sum_{j' < j} tot[j'][e]
@@ -135,6 +141,93 @@ assign_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int
     }
 }
 
+// A shard of a batch split over several GPUs (contiguous token ranges, in rank
+// order).  base[j][e] is the queue place, in the whole batch, of this shard's
+// first j-th choice of expert e; it comes from every shard's counts, exchanged
+// once (shard_base_kernel).  C is the whole batch's capacity.  A (t, j) is kept
+// iff its place in the whole batch, base[j][e] + its place among this shard's
+// j-th choices of e, is below C, which is the unsharded rule.  Kept rows are
+// numbered per expert inside the shard (choice rank first, then token order),
+// so the shard's gathered rows, expert FFN and combine work unchanged.
+__global__ void __launch_bounds__(kDispatchTB)
+assign_shard_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int64_t C,
+                    const int32_t *__restrict__ hist_excl /* [nblk][k][E] */,
+                    const int32_t *__restrict__ tot /* [k][E] this shard's totals */,
+                    const int32_t *__restrict__ base /* [k][E] */, int32_t *__restrict__ slot,
+                    int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+    extern __shared__ int32_t a_smem[];
+    int32_t *warp_cnt = a_smem;                                // [warps][E]
+    int32_t *kept_before = warp_cnt + kDispatchWarps * E;      // [E] kept rows of choices < j
+    int32_t *offs = kept_before + E;                           // [E + 1]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchTB + tid;
+    auto kept_of = [&](int j, int e) -> int32_t {  // kept j-th choices of e in this shard
+        const int64_t room = C - static_cast<int64_t>(base[j * E + e]);
+        const int64_t n = tot[j * E + e];
+        return static_cast<int32_t>(room <= 0 ? 0 : (room < n ? room : n));
+    };
+    for (int e = tid; e < E; e += blockDim.x) {
+        int32_t total = 0;
+        for (int j = 0; j < k; ++j) total += kept_of(j, e);
+        offs[e] = total;
+        kept_before[e] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int32_t run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t c = offs[e];
+            offs[e] = run;
+            run += c;
+            if (blockIdx.x == 0) counts[e] = c;
+        }
+        offs[E] = run;
+        if (blockIdx.x == 0)
+            for (int e = 0; e <= E; ++e) offsets[e] = offs[e];
+    }
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+        for (int i = tid; i < kDispatchWarps * E; i += blockDim.x) warp_cnt[i] = 0;
+        __syncthreads();
+        int e = -1;
+        if (t < N) {
+            e = topk_idx[t * k + j];
+            if (e < 0 || e >= E) e = -1;
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank_in_warp = __popc(same & lt_mask);
+        if (e >= 0 && rank_in_warp == 0) warp_cnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        if (e >= 0) {
+            int64_t local = static_cast<int64_t>(hist_excl[(static_cast<int64_t>(blockIdx.x) * k + j) * E + e]) +
+                            rank_in_warp;
+            for (int w = 0; w < warp; ++w) local += warp_cnt[w * E + e];
+            const int64_t place = static_cast<int64_t>(base[j * E + e]) + local;
+            slot[t * k + j] = place < C ? static_cast<int32_t>(kept_before[e] + local) : -1;
+        } else if (t < N) {
+            slot[t * k + j] = -1;
+        }
+        __syncthreads();
+        for (int ee = tid; ee < E; ee += blockDim.x) kept_before[ee] += kept_of(j, ee);
+        __syncthreads();
+    }
+}
+
+// base[j][e] = sum over all shards of the choices j' < j of e, plus the j-th
+// choices of e in the shards before `rank`.  One thread per (j, e).
+__global__ void shard_base_kernel(const int32_t *__restrict__ all_counts /* [G][k][E] */, int G, int rank,
+                                  int E, int k, int32_t *__restrict__ base) {
+    const int pair = blockIdx.x * blockDim.x + threadIdx.x;
+    if (pair >= k * E) return;
+    const int j = pair / E, e = pair % E;
+    int64_t b = 0;
+    for (int jj = 0; jj < j; ++jj)
+        for (int g = 0; g < G; ++g) b += all_counts[(static_cast<int64_t>(g) * k + jj) * E + e];
+    for (int g = 0; g < rank; ++g) b += all_counts[(static_cast<int64_t>(g) * k + j) * E + e];
+    base[pair] = static_cast<int32_t>(b);
+}
+
 // The whole slot assignment for a batch of at most kSmallTB tokens in one
 // block: count per (j, e), then place each (t, j) in token order within its
 // choice rank (warp match + per-warp counts), as in the multi-block passes.
@@ -145,6 +238,8 @@ __global__ void __launch_bounds__(kSmallTB)
 dispatch_small_kernel(const int32_t *__restrict__ topk_idx, int64_t N, int E, int k, int64_t C,
                       int32_t *__restrict__ slot, int32_t *__restrict__ counts,
                       int32_t *__restrict__ offsets) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ int32_t s_smem[];
     int32_t *tot = s_smem;                         // [k][E]
     int32_t *warp_cnt = tot + k * E;               // [warps][E]
@@ -214,6 +309,8 @@ __global__ void __launch_bounds__(256)
 gather_kernel(const U *__restrict__ x, int64_t units_per_row, const int32_t *__restrict__ topk_idx,
               const int32_t *__restrict__ slot, const int32_t *__restrict__ offsets, int64_t Nk, int k,
               U *__restrict__ xg) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = Nk * units_per_row;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -257,22 +354,64 @@ cudaError_t launch_dispatch(const int32_t *topk_idx, const void *x, int elem_byt
     }
     const size_t small_smem = sizeof(int32_t) * (static_cast<size_t>(k) * E + kSmallWarps * E + E + E + 1);
     if (dispatch_single_block(N, E, k)) {
-        dispatch_small_kernel<<<1, kSmallTB, small_smem, s>>>(topk_idx, N, E, k, C, slot, counts, offsets);
+        cudaError_t e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(kSmallTB), small_smem, s, topk_idx, N, E, k,
+                                   C, slot, counts, offsets);
+        if (e != cudaSuccess) return e;
     } else {
         const int64_t nblk = dispatch_blocks(N);
         int32_t *hist = static_cast<int32_t *>(ws);
         int32_t *tot = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) +
                                                    align_up(sizeof(int32_t) * static_cast<size_t>(nblk) * k * E, 256));
-        hist_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, sizeof(int32_t) * E, s>>>(topk_idx, N, E,
-                                                                                         k, hist);
+        cudaError_t e = launch_pdl(hist_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kDispatchTB),
+                                   sizeof(int32_t) * E, s, topk_idx, N, E, k, hist);
+        if (e != cudaSuccess) return e;
         const int pairs = k * E;
         const int warps_per_block = 8;
-        scan_kernel<<<(pairs + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, s>>>(
-            hist, static_cast<int>(nblk), E, k, tot);
+        e = launch_pdl(scan_kernel, dim3((pairs + warps_per_block - 1) / warps_per_block), dim3(warps_per_block * 32),
+                       0, s, hist, static_cast<int>(nblk), E, k, tot);
+        if (e != cudaSuccess) return e;
         const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kDispatchWarps) * E + E + E + 1);
-        assign_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, smem, s>>>(topk_idx, N, E, k, C, hist, tot,
-                                                                            slot, counts, offsets);
+        e = launch_pdl(assign_kernel, dim3(static_cast<unsigned>(nblk)), dim3(kDispatchTB), smem, s, topk_idx, N, E,
+                       k, C, static_cast<const int32_t *>(hist), static_cast<const int32_t *>(tot), slot, counts,
+                       offsets);
+        if (e != cudaSuccess) return e;
     }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_gather(topk_idx, slot, offsets, x, elem_bytes, N, d, k, x_gathered, s);
+}
+
+cudaError_t launch_shard_count(const int32_t *topk_idx, int64_t N, int E, int k, int32_t *counts_je,
+                               void *ws, cudaStream_t s) {
+    if (N == 0) return cudaMemsetAsync(counts_je, 0, sizeof(int32_t) * k * E, s);
+    const int64_t nblk = dispatch_blocks(N);
+    int32_t *hist = static_cast<int32_t *>(ws);
+    hist_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, sizeof(int32_t) * E, s>>>(topk_idx, N, E, k, hist);
+    const int pairs = k * E;
+    scan_kernel<<<(pairs + 7) / 8, 256, 0, s>>>(hist, static_cast<int>(nblk), E, k, counts_je);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shard_base(const int32_t *all_counts, int G, int rank, int E, int k, int32_t *base,
+                              cudaStream_t s) {
+    const int pairs = k * E;
+    shard_base_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(all_counts, G, rank, E, k, base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shard_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N, int d,
+                                  int E, int k, int64_t C, const int32_t *counts_je, const int32_t *base,
+                                  int32_t *slot, int32_t *counts, int32_t *offsets, void *x_gathered,
+                                  void *ws, cudaStream_t s) {
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s);
+        return e;
+    }
+    const int64_t nblk = dispatch_blocks(N);
+    const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kDispatchWarps) * E + E + E + 1);
+    assign_shard_kernel<<<static_cast<unsigned>(nblk), kDispatchTB, smem, s>>>(
+        topk_idx, N, E, k, C, static_cast<const int32_t *>(ws), counts_je, base, slot, counts, offsets);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_gather(topk_idx, slot, offsets, x, elem_bytes, N, d, k, x_gathered, s);
@@ -293,13 +432,12 @@ cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const in
     if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
     if (blocks < 1) blocks = 1;
     if (vec16)
-        gather_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            static_cast<const uint4 *>(x), units, topk_idx, slot, offsets, Nk, k, static_cast<uint4 *>(x_gathered));
-    else
-        gather_kernel<uint16_t><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            static_cast<const uint16_t *>(x), units, topk_idx, slot, offsets, Nk, k,
-            static_cast<uint16_t *>(x_gathered));
-    return cudaGetLastError();
+        return launch_pdl(gather_kernel<uint4>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                          static_cast<const uint4 *>(x), units, topk_idx, slot, offsets, Nk, k,
+                          static_cast<uint4 *>(x_gathered));
+    return launch_pdl(gather_kernel<uint16_t>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                      static_cast<const uint16_t *>(x), units, topk_idx, slot, offsets, Nk, k,
+                      static_cast<uint16_t *>(x_gathered));
 }
 
 }  // namespace moe

@@ -6,7 +6,7 @@
 // mantissa bits and miss the fp32 tolerance) and for bf16 shapes whose rows
 // are not 16-byte multiples (tensor-memory copies need them).
 //
-// out[r, n] = act( sum_k A[r, k] * W[e, n, k] )  for the rows r of expert e,
+// out[r, n] = act( sum_k A[r, k] * W[e, n, k] + bias[e, n] )  for the rows r of expert e,
 // with A and W K-major.  Tiles of 64 rows x 64 outputs; rows are grouped per
 // expert using the device-side counts/offsets, so no host synchronisation.
 #include "common.cuh"
@@ -18,10 +18,14 @@ namespace {
 
 constexpr int TM = 64, TN = 64, TK = 16;
 
-template <typename T, bool RELU>
+// act: 0 none, 1 ReLU, 2 GELU (x * Phi(x)); bias [E][Nw] fp32 or null.
+template <typename T>
 __global__ void __launch_bounds__(256)
 simt_gemm_kernel(const T *__restrict__ A, const T *__restrict__ W, const int32_t *__restrict__ offsets,
-                 const int32_t *__restrict__ counts, int E, int Nw, int K, T *__restrict__ out) {
+                 const int32_t *__restrict__ counts, int E, int Nw, int K, T *__restrict__ out,
+                 const float *__restrict__ bias, int act) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int32_t tile_prefix[257];
     __shared__ float As[TK][TM + 1];
     __shared__ float Ws[TK][TN + 1];
@@ -82,7 +86,9 @@ simt_gemm_kernel(const T *__restrict__ A, const T *__restrict__ W, const int32_t
             const int n = n0 + tx * 4 + j;
             if (n >= Nw) continue;
             float v = acc[i][j];
-            if (RELU) v = fmaxf(v, 0.0f);
+            if (bias) v += bias[static_cast<int64_t>(e) * Nw + n];
+            if (act == 2) v = 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+            else if (act == 1) v = fmaxf(v, 0.0f);
             out[(row0 + r) * Nw + n] = from_f32<T>(v);
         }
     }
@@ -91,27 +97,31 @@ simt_gemm_kernel(const T *__restrict__ A, const T *__restrict__ W, const int32_t
 template <typename T>
 cudaError_t launch_simt_ffn_t(const void *xg, const int32_t *offsets, const int32_t *counts,
                               const void *W_up, const void *W_down, int64_t rows, int d, int d_ff,
-                              int E, void *out, void *H, cudaStream_t s) {
+                              int E, void *out, void *H, cudaStream_t s, int act, const float *b_up,
+                              const float *b_down) {
     const int64_t mtiles = (rows + TM - 1) / TM + E;  // upper bound on sum_e ceil(counts[e] / TM)
     if (mtiles > 65535) return cudaErrorInvalidConfiguration;
     dim3 g_up((d_ff + TN - 1) / TN, static_cast<unsigned>(mtiles));
-    simt_gemm_kernel<T, true><<<g_up, 256, 0, s>>>(static_cast<const T *>(xg), static_cast<const T *>(W_up),
-                                                   offsets, counts, E, d_ff, d, static_cast<T *>(H));
+    cudaError_t e = launch_pdl(simt_gemm_kernel<T>, g_up, dim3(256), 0, s, static_cast<const T *>(xg),
+                               static_cast<const T *>(W_up), offsets, counts, E, d_ff, d, static_cast<T *>(H), b_up,
+                               act);
+    if (e != cudaSuccess) return e;
     dim3 g_dn((d + TN - 1) / TN, static_cast<unsigned>(mtiles));
-    simt_gemm_kernel<T, false><<<g_dn, 256, 0, s>>>(static_cast<const T *>(H), static_cast<const T *>(W_down),
-                                                    offsets, counts, E, d, d_ff, static_cast<T *>(out));
-    return cudaGetLastError();
+    return launch_pdl(simt_gemm_kernel<T>, g_dn, dim3(256), 0, s, static_cast<const T *>(H),
+                      static_cast<const T *>(W_down), offsets, counts, E, d, d_ff, static_cast<T *>(out), b_down, 0);
 }
 
 }  // namespace
 
 cudaError_t launch_simt_ffn(const void *xg, const int32_t *offsets, const int32_t *counts,
                             const void *W_up, const void *W_down, int dt, int64_t rows, int d,
-                            int d_ff, int E, void *out, void *H, cudaStream_t s) {
+                            int d_ff, int E, void *out, void *H, cudaStream_t s, int act,
+                            const float *b_up, const float *b_down) {
     if (dt == 1)
         return launch_simt_ffn_t<__nv_bfloat16>(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E,
-                                                out, H, s);
-    return launch_simt_ffn_t<float>(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E, out, H, s);
+                                                out, H, s, act, b_up, b_down);
+    return launch_simt_ffn_t<float>(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E, out, H, s, act,
+                                    b_up, b_down);
 }
 
 }  // namespace moe

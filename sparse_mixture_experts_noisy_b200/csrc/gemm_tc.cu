@@ -44,7 +44,10 @@ constexpr int kBM = 128;       // MMA M
 constexpr int kBK = 64;        // K elements per stage (128 bytes of bf16 = one swizzle row)
 constexpr int kThreads = 192;
 
-enum { EPI_BF16 = 0, EPI_BF16_RELU = 1, EPI_F32 = 2 };
+// Epilogues: bf16 out with the optional bias (down projection), bf16 out with
+// bias and activation (up projection), raw fp32 partial sums (K splits; bias
+// and activation are applied once the splits are added).
+enum { EPI_BF16 = 0, EPI_BF16_ACT = 1, EPI_F32 = 2 };
 
 struct TcArgs {
     const int32_t *offsets;
@@ -55,7 +58,38 @@ struct TcArgs {
     int64_t split_stride;  // elements between K-split partial buffers (EPI_F32)
     uint32_t *status;
     uint64_t timeout_ns;
+    const float *bias;  // [E][Nw] fp32 or null: added to every output row of expert e
+    int act;            // EPI_BF16_ACT: 1 = ReLU, 2 = GELU (x * Phi(x))
 };
+
+__device__ __forceinline__ float activate(float v, int act) {
+    if (act == 2) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+    return fmaxf(v, 0.0f);
+}
+
+// Bias and activation for one 32-column chunk of TMEM values.  Token-row tiles
+// (swap = false): columns are weight rows col0..col0+31, the same for all lanes.
+// Weight-row tiles (swap = true): the lane's weight row w is fixed.
+template <int EPI, bool SWAP>
+__device__ __forceinline__ void bias_act(uint32_t (&r)[32], const TcArgs &args, int e, int col0, int w) {
+    if (EPI == EPI_F32) return;
+    if (args.bias != nullptr) {
+        const float *b = args.bias + static_cast<int64_t>(e) * args.Nw;
+        if (SWAP) {
+            const float bw = (w < args.Nw) ? b[w] : 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + bw);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < args.Nw) r[i] = __float_as_uint(__uint_as_float(r[i]) + b[col0 + i]);
+        }
+    }
+    if (EPI == EPI_BF16_ACT) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(activate(__uint_as_float(r[i]), args.act));
+    }
+}
 
 template <int BN>
 __host__ __device__ constexpr uint32_t tmem_cols() {
@@ -140,18 +174,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
     const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
     const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
 
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
-    __syncthreads();
+    pdl_trigger();
     if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            pre_s[e] = run;
-            const int c = cnt_s[e];
-            const int units = SWAP ? ((Nw + kBM - 1) / kBM) * ((c + BN - 1) / BN)
-                                   : ((c + kBM - 1) / kBM) * ((Nw + BN - 1) / BN);
-            run += units * splits;
-        }
-        pre_s[E] = run;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
@@ -170,6 +194,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
     if (warp == 1) {
         tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
         tmem_relinquish();
+    }
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            pre_s[e] = run;
+            const int c = cnt_s[e];
+            const int units = SWAP ? ((Nw + kBM - 1) / kBM) * ((c + BN - 1) / BN)
+                                   : ((c + kBM - 1) / kBM) * ((Nw + BN - 1) / BN);
+            run += units * splits;
+        }
+        pre_s[E] = run;
     }
     tc_fence_before();
     __syncthreads();
@@ -297,11 +335,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, r);
                 tmem_wait_ld();
-                if (EPI == EPI_BF16_RELU) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
-                }
+                bias_act<EPI, SWAP>(r, args, t.e, t.w0 + c * 32, t.w0 + row_in_tile);
                 if (!SWAP) {
                     const bool rv = t.tok0 + row_in_tile < cnt;
                     const int64_t grow = row_base + t.tok0 + row_in_tile;
@@ -413,15 +447,8 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     const uint32_t full0_lead = map_to_cta(full0, 0);
     const uint32_t tempty0_lead = map_to_cta(tempty0, 0);
 
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
-    __syncthreads();
+    pdl_trigger();
     if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            pre_s[e] = run;
-            run += ((cnt_s[e] + BT - 1) / BT) * ((Nw + BT - 1) / BT) * splits;
-        }
-        pre_s[E] = run;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
@@ -440,6 +467,17 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(&tmem_holder), TMEM_COLS);
         tmem_relinquish_pair();
+    }
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = args.counts[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            pre_s[e] = run;
+            run += ((cnt_s[e] + BT - 1) / BT) * ((Nw + BT - 1) / BT) * splits;
+        }
+        pre_s[E] = run;
     }
     tc_fence_before();
     __syncthreads();
@@ -582,10 +620,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, r);
                 tmem_wait_ld();
-                if (EPI == EPI_BF16_RELU) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
-                }
+                bias_act<EPI, false>(r, args, e, w0 + c * 32, 0);
                 const int col0 = w0 + c * 32;
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo;
 #pragma unroll
@@ -664,7 +699,7 @@ template <int BN, bool SWAP, int EPI, int STAGES>
 cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
                       const int32_t *offsets, const int32_t *counts, int splits, void *out,
                       int64_t ldo, int64_t split_stride, uint32_t *status, uint64_t timeout_ns,
-                      int grid, cudaStream_t s) {
+                      int grid, cudaStream_t s, const float *bias = nullptr, int act = 1) {
     CUtensorMap tm_tok, tm_w;
     if (!make_map_2d(&tm_tok, tok, tok_rows, K, SWAP ? BN : kBM)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tm_w, W, E, Nw, K, SWAP ? kBM : BN)) return cudaErrorInvalidValue;
@@ -676,15 +711,15 @@ cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, i
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns};
-    kern<<<grid, kThreads, smem, s>>>(tm_tok, tm_w, a);
-    return cudaGetLastError();
+    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act};
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, tm_tok, tm_w, a);
 }
 
 template <int EPI, int STAGES>
 cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
                        const int32_t *offsets, const int32_t *counts, void *out, int64_t ldo,
-                       uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s) {
+                       uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
+                       const float *bias = nullptr, int act = 1) {
     CUtensorMap tm_tok, tm_w;
     if (!make_map_2d(&tm_tok, tok, tok_rows, K, 128)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
@@ -703,24 +738,43 @@ cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, 
         max_clusters < pairs)
         pairs = max_clusters;
     (void)cudaGetLastError();
-    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns};
-    kern<<<2 * pairs, kThreads, smem, s>>>(tm_tok, tm_w, a);
-    return cudaGetLastError();
+    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns, bias, act};
+    return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), smem, s, tm_tok, tm_w, a);
 }
 
-// Sum of K-split fp32 partials into dtype rows, in split order.
+// Sum of K-split fp32 partials into bf16 rows, in split order, then the
+// expert's bias (nullable, [E][d]) and the activation (0 none, 1 ReLU,
+// 2 GELU).  Only the kept rows (below offsets[E]) are touched.
 __global__ void __launch_bounds__(256)
 reduce_parts_kernel(const float *__restrict__ parts, int nparts, int64_t part_stride,
-                    const int32_t *__restrict__ offsets, int E, int d,
-                    __nv_bfloat16 *__restrict__ out) {
+                    const int32_t *__restrict__ offsets, int E, int d, const float *__restrict__ bias,
+                    int act, __nv_bfloat16 *__restrict__ out) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t rows = offsets[E];
-    const int64_t total = rows * (d / 4);
+    const int q = d / 4;
+    const int64_t total = rows * q;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float4 a = reinterpret_cast<const float4 *>(parts)[i];
         for (int p = 1; p < nparts; ++p) {
             const float4 b = reinterpret_cast<const float4 *>(parts + p * part_stride)[i];
             a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        if (bias != nullptr) {
+            const int64_t row = i / q;
+            const int c = static_cast<int>(i - row * q) * 4;
+            int lo = 0, hi = E;  // offsets[lo] <= row < offsets[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (offsets[mid] <= row) lo = mid; else hi = mid;
+            }
+            const float4 bb = *reinterpret_cast<const float4 *>(bias + static_cast<int64_t>(lo) * d + c);
+            a.x += bb.x; a.y += bb.y; a.z += bb.z; a.w += bb.w;
+        }
+        if (act != 0) {
+            a.x = activate(a.x, act); a.y = activate(a.y, act);
+            a.z = activate(a.z, act); a.w = activate(a.w, act);
         }
         __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(out) + 2 * i;
         o[0] = __floats2bfloat162_rn(a.x, a.y);
@@ -730,9 +784,20 @@ reduce_parts_kernel(const float *__restrict__ parts, int nparts, int64_t part_st
 
 }  // namespace
 
+// K splits that give about `waves` units per SM for `units` equal tiles.
+int decode_splits(int64_t units, int K, int num_sms, int64_t waves) {
+    const int kb_total = (K + kBK - 1) / kBK;
+    int s = static_cast<int>((waves * num_sms + units - 1) / units);
+    if (s > 8) s = 8;
+    if (s > kb_total) s = kb_total;
+    if (s < 1) s = 1;
+    return s;
+}
+
 TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
     TcPlan p{};
     p.decode = rows <= 256;
+    p.splits_up = 1;
     p.splits_down = 1;
     // CTA-pair tiles for prefill; MOE_TC_PAIR=0 selects the one-CTA tiles
     static const int pair_env = [] {
@@ -741,13 +806,11 @@ TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
     }();
     p.pair = !p.decode && pair_env != 0 && num_sms >= 2;
     if (p.decode) {
-        const int64_t units = static_cast<int64_t>(E) * ((d + kBM - 1) / kBM);
-        const int kb_total = (d_ff + kBK - 1) / kBK;
-        int s = static_cast<int>((6LL * num_sms + units - 1) / units);
-        if (s > 8) s = 8;
-        if (s > kb_total) s = kb_total;
-        if (s < 1) s = 1;
-        p.splits_down = s;
+        // weight-streaming tiles: enough equal units that the last wave is a
+        // small part of the whole, split over K (fp32 partials) to get there
+        // (the combine reads every down partial, so that one aims lower)
+        p.splits_up = decode_splits(static_cast<int64_t>(E) * ((d_ff + kBM - 1) / kBM), d, num_sms, 12);
+        p.splits_down = decode_splits(static_cast<int64_t>(E) * ((d + kBM - 1) / kBM), d_ff, num_sms, 6);
     }
     return p;
 }
@@ -755,34 +818,57 @@ TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
 size_t tc_ffn_ws_bytes(int64_t rows, int d, int d_ff, int E, int num_sms) {
     const TcPlan p = plan_tc_ffn(rows, d, d_ff, E, num_sms);
     size_t b = align_up(static_cast<size_t>(rows) * d_ff * 2, 256);  // hidden activations
-    if (p.decode) b += align_up(static_cast<size_t>(p.splits_down) * rows * d * 4, 256);
+    if (p.decode) {
+        b += align_up(static_cast<size_t>(p.splits_down) * rows * d * 4, 256);
+        if (p.splits_up > 1) b += align_up(static_cast<size_t>(p.splits_up) * rows * d_ff * 4, 256);
+    }
     return b;
+}
+
+int tc_ffn_launches(const TcPlan &p, bool combine_reads_parts) {
+    if (!p.decode) return 2;
+    return 2 + (p.splits_up > 1 ? 1 : 0) + (combine_reads_parts ? 0 : 1);
 }
 
 cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t *counts,
                           const void *W_up, const void *W_down, int64_t rows, int d, int d_ff,
                           int E, void *out, void *H, float *parts, bool combine_reads_parts,
                           uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
-                          TcPlan *plan_out) {
+                          TcPlan *plan_out, int act, const float *b_up, const float *b_down) {
     const TcPlan p = plan_tc_ffn(rows, d, d_ff, E, num_sms);
     if (plan_out) *plan_out = p;
     cudaError_t e;
     if (!p.decode && p.pair) {
-        e = launch_tc2<EPI_BF16_RELU, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
-                                         timeout_ns, num_sms, s);
+        e = launch_tc2<EPI_BF16_ACT, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
+                                        timeout_ns, num_sms, s, b_up, act);
         if (e != cudaSuccess) return e;
         return launch_tc2<EPI_BF16, 6>(H, rows, W_down, E, d, d_ff, offsets, counts, out, d, status,
-                                       timeout_ns, num_sms, s);
+                                       timeout_ns, num_sms, s, b_down, 0);
     }
     if (!p.decode) {
-        e = launch_tc<256, false, EPI_BF16_RELU, 4>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H,
-                                                    d_ff, 0, status, timeout_ns, num_sms, s);
+        e = launch_tc<256, false, EPI_BF16_ACT, 4>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H,
+                                                   d_ff, 0, status, timeout_ns, num_sms, s, b_up, act);
         if (e != cudaSuccess) return e;
         return launch_tc<256, false, EPI_BF16, 4>(H, rows, W_down, E, d, d_ff, offsets, counts, 1, out,
-                                                  d, 0, status, timeout_ns, num_sms, s);
+                                                  d, 0, status, timeout_ns, num_sms, s, b_down, 0);
     }
-    e = launch_tc<64, true, EPI_BF16_RELU, 8>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H, d_ff,
-                                              0, status, timeout_ns, num_sms, s);
+    if (p.splits_up > 1) {
+        // up projection split over K into fp32 partials, then ReLU of their sum
+        float *parts_up = parts + align_up(static_cast<size_t>(p.splits_down) * rows * d * 4, 256) / 4;
+        const int64_t ustride = rows * static_cast<int64_t>(d_ff);
+        e = launch_tc<64, true, EPI_F32, 8>(xg, rows, W_up, E, d_ff, d, offsets, counts, p.splits_up, parts_up,
+                                            d_ff, ustride, status, timeout_ns, num_sms, s);
+        if (e != cudaSuccess) return e;
+        const int64_t total_h = rows * (d_ff / 4);
+        const int hblocks =
+            static_cast<int>((total_h + 255) / 256 < 4 * num_sms ? (total_h + 255) / 256 : 4 * num_sms);
+e = launch_pdl(reduce_parts_kernel, dim3(hblocks > 0 ? hblocks : 1), dim3(256), 0, s,
+                       static_cast<const float *>(parts_up), p.splits_up, ustride,
+                       static_cast<const int32_t *>(offsets), E, d_ff, b_up, act, static_cast<__nv_bfloat16 *>(H));
+    } else {
+        e = launch_tc<64, true, EPI_BF16_ACT, 8>(xg, rows, W_up, E, d_ff, d, offsets, counts, 1, H, d_ff, 0,
+                                                 status, timeout_ns, num_sms, s, b_up, act);
+    }
     if (e != cudaSuccess) return e;
     const int64_t pstride = rows * static_cast<int64_t>(d);
     e = launch_tc<64, true, EPI_F32, 8>(H, rows, W_down, E, d, d_ff, offsets, counts, p.splits_down,
@@ -790,9 +876,9 @@ cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t 
     if (e != cudaSuccess || combine_reads_parts) return e;
     const int64_t total = rows * (d / 4);
     const int blocks = static_cast<int>((total + 255) / 256 < 4 * num_sms ? (total + 255) / 256 : 4 * num_sms);
-    reduce_parts_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(parts, p.splits_down, pstride, offsets, E, d,
-                                                                static_cast<__nv_bfloat16 *>(out));
-    return cudaGetLastError();
+    return launch_pdl(reduce_parts_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s,
+                      static_cast<const float *>(parts), p.splits_down, pstride, static_cast<const int32_t *>(offsets),
+                      E, d, b_down, 0, static_cast<__nv_bfloat16 *>(out));
 }
 
 // Diagnostic: one CTA waits on a barrier that nothing completes.

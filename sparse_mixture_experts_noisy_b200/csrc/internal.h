@@ -9,6 +9,25 @@ namespace moe {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch with programmatic dependent launch allowed: the kernel may be
+// scheduled while the previous kernel on the stream finishes; it must call
+// pdl_wait() before touching anything that kernel produces or reads.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Router (route.cu).  status (nullable) is zeroed by the first block.
 cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b_g,
                          const float *noise, float sigma, int64_t N, int d, int E, int k,
@@ -23,37 +42,54 @@ size_t dispatch_ws_bytes(int64_t N, int E, int k);
 cudaError_t launch_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N,
                             int d, int E, int k, int64_t C, int32_t *slot, int32_t *counts,
                             int32_t *offsets, void *x_gathered, void *ws, cudaStream_t s);
+// Token-sharded batches (one exchange of per-(choice, expert) counts).
+cudaError_t launch_shard_count(const int32_t *topk_idx, int64_t N, int E, int k, int32_t *counts_je,
+                               void *ws, cudaStream_t s);
+cudaError_t launch_shard_base(const int32_t *all_counts, int G, int rank, int E, int k, int32_t *base,
+                              cudaStream_t s);
+cudaError_t launch_shard_dispatch(const int32_t *topk_idx, const void *x, int elem_bytes, int64_t N, int d,
+                                  int E, int k, int64_t C, const int32_t *counts_je, const int32_t *base,
+                                  int32_t *slot, int32_t *counts, int32_t *offsets, void *x_gathered,
+                                  void *ws, cudaStream_t s);
 cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const int32_t *offsets,
                           const void *x, int elem_bytes, int64_t N, int d, int k, void *x_gathered,
                           cudaStream_t s);
 
 // Combine (combine.cu).  Either out_rows (dtype rows, nparts == 0) or nparts
 // fp32 partial buffers `part_stride` elements apart.
+// b_down (nullable, [E][d]) is added to the summed partials (nparts > 0 only;
+// dtype rows already carry it).
 cudaError_t launch_combine(const void *out_rows, const float *parts, int nparts,
                            int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
                            const int32_t *offsets, const float *gates, int dt, int64_t N, int d,
-                           int k, int E, void *y, cudaStream_t s);
+                           int k, int E, void *y, cudaStream_t s, const float *b_down = nullptr);
 
 // CUDA-core expert FFN (ffn_simt.cu).  H: [rows, d_ff] of dtype.
+// act: 1 = ReLU, 2 = GELU; b_up [E][d_ff], b_down [E][d] fp32, nullable.
 cudaError_t launch_simt_ffn(const void *xg, const int32_t *offsets, const int32_t *counts,
                             const void *W_up, const void *W_down, int dt, int64_t rows, int d,
-                            int d_ff, int E, void *out, void *H, cudaStream_t s);
+                            int d_ff, int E, void *out, void *H, cudaStream_t s, int act = 1,
+                            const float *b_up = nullptr, const float *b_down = nullptr);
 
 // Tensor-core expert FFN (gemm_tc.cu).
 struct TcPlan {
     bool decode;      // weight rows as the MMA's M (few tokens per expert)
     bool pair;        // prefill on CTA pairs (tcgen05 cta_group::2)
+    int splits_up;    // K splits of the up projection (decode only; > 1 adds a ReLU-sum pass)
     int splits_down;  // K splits of the down projection (decode only)
 };
 TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms);
 size_t tc_ffn_ws_bytes(int64_t rows, int d, int d_ff, int E, int num_sms);
-// H: [rows, d_ff] bf16; parts: splits x [rows, d] fp32 (decode plan only).  With
+int tc_ffn_launches(const TcPlan &p, bool combine_reads_parts);
+// H: [rows, d_ff] bf16; parts: splits_down x [rows, d] fp32 then, if
+// splits_up > 1, splits_up x [rows, d_ff] fp32 (decode plan only).  With
 // combine_reads_parts the decode plan leaves the partials for the combine.
 cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t *counts,
                           const void *W_up, const void *W_down, int64_t rows, int d, int d_ff,
                           int E, void *out, void *H, float *parts, bool combine_reads_parts,
                           uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
-                          TcPlan *plan_out);
+                          TcPlan *plan_out, int act = 1, const float *b_up = nullptr,
+                          const float *b_down = nullptr);
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
 
 }  // namespace moe

@@ -6,9 +6,9 @@
 // -inf scatter, softmax).
 //
 // The dot products run on CUDA cores in fp32 (fmaf).  Two launch shapes:
-// large batches give one token to each lane (W_g loads are then warp-wide
-// broadcasts, registers stay few and occupancy high), small batches give one
-// token to a whole block so that even 64 tokens spread over the GPU.  The bias
+// large batches give 4 tokens to each warp with W_g staged in shared memory,
+// small batches give one token to a whole block so that even 64 tokens spread
+// over the GPU.  The bias
 // and the noise are added with explicit round-to-nearest adds and multiplies,
 // so the compiler cannot fuse the noise step into one rounding.
 #include "common.cuh"
@@ -75,99 +75,165 @@ __device__ __forceinline__ float add_noise(float s, float sigma, float eps) {
 }
 
 // ------------------------------------------------------------------ large batches
-// Lane = token: a block of 4 warps owns 32 tokens; warp w adds up the products of
-// its quarter of d, lane by lane, while every lane of the warp reads the same
-// W_g entries (broadcast loads that L1 serves once per warp).  The four partial
-// sums of a (token, expert) are added in warp order through shared memory.
-// Each lane then picks its token's k experts over the E scores and forms the
-// softmax.
-constexpr int kLaneWarps = 4;
+// A block of 8 warps owns 32 tokens, 4 per warp.  For each 512-wide chunk of
+// d the block stages W_g[e0 .. e0+8)[chunk] in shared memory; the lanes of a
+// warp read 16-byte pieces of their 4 tokens' rows (consecutive lanes,
+// consecutive bytes) and keep 4 tokens x 8 experts of fp32 partial sums, which
+// the warp adds with shuffles once d is done.  Then the warp picks each
+// token's k experts (rounds of a warp-wide arg-max) and forms the softmax.
+constexpr int kTileWarps = 8;
+constexpr int kTileTPW = 4;                    // tokens per warp
+constexpr int kTileTok = kTileWarps * kTileTPW;
+constexpr int kTileDC = 512;                   // d chunk staged per pass
+constexpr int kTileEC = 8;                     // experts per pass
 
-template <typename T, int VEC, int EC>
-__global__ void __launch_bounds__(kLaneWarps * 32)
-route_lanes_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
-                   const float *__restrict__ b_g, const float *__restrict__ noise, float sigma,
-                   int64_t N, int d, int E, int k, float *__restrict__ logits_out,
-                   int32_t *__restrict__ topk_idx, float *__restrict__ gates,
-                   uint32_t *__restrict__ status) {
+template <typename T, int VEC>
+__global__ void __launch_bounds__(kTileWarps * 32)
+route_tile_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
+                  const float *__restrict__ b_g, const float *__restrict__ noise, float sigma,
+                  int64_t N, int d, int E, int k, float *__restrict__ logits_out,
+                  int32_t *__restrict__ topk_idx, float *__restrict__ gates,
+                  uint32_t *__restrict__ status) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ float route_smem[];
-    float *part = route_smem;                          // [4 warps][32 lanes][EC + 1]
-    float *sc = part + kLaneWarps * 32 * (EC + 1);     // [32 lanes][E + 1]
+    float *ws = route_smem;                               // [kTileEC][kTileDC]
+    float *s_sc = ws + kTileEC * kTileDC;                  // [kTileTok][E]
+    float *pick_v = s_sc + static_cast<size_t>(kTileTok) * E + static_cast<size_t>(threadIdx.x >> 5) * 2 * k;
+    int *pick_e = reinterpret_cast<int *>(pick_v + k);
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * 32 + lane;
-    const bool live = t < N;
-    const int steps = (d + VEC - 1) / VEC;
-    const int i_lo = static_cast<int>(static_cast<int64_t>(warp) * steps / kLaneWarps) * VEC;
-    const int i_hi = min(d, static_cast<int>(static_cast<int64_t>(warp + 1) * steps / kLaneWarps) * VEC);
-    const T *xr = x + (live ? t : 0) * static_cast<int64_t>(d);
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileTok + warp * kTileTPW;
+    const int ntok = (t0 >= N) ? 0 : ((N - t0 < kTileTPW) ? static_cast<int>(N - t0) : kTileTPW);
+    const bool vec_w = (d % 4 == 0) && (reinterpret_cast<uintptr_t>(W_g) % 16 == 0);
 
-    for (int e0 = 0; e0 < E; e0 += EC) {
-        float acc[EC];
+    for (int e0 = 0; e0 < E; e0 += kTileEC) {
+        float acc[kTileTPW][kTileEC];
 #pragma unroll
-        for (int c = 0; c < EC; ++c) acc[c] = 0.0f;
-        if (live) {
-            for (int i = i_lo; i < i_hi; i += VEC) {
-                float xv[VEC];
-                XLoad<T, VEC>::load(xr + i, xv);
+        for (int a = 0; a < kTileTPW; ++a)
 #pragma unroll
-                for (int c = 0; c < EC; ++c) {
-                    if (e0 + c < E) {
+            for (int c = 0; c < kTileEC; ++c) acc[a][c] = 0.0f;
+        for (int dc = 0; dc < d; dc += kTileDC) {
+            const int dn = min(kTileDC, d - dc);
+            __syncthreads();
+            if (vec_w) {
+                // 16-byte pieces, every one of the thread's loads in flight at once
+                constexpr int kPieces = kTileEC * kTileDC / 4 / (kTileWarps * 32);
+                float4 tmp[kPieces];
+#pragma unroll
+                for (int u = 0; u < kPieces; ++u) {
+                    const int i = (threadIdx.x + u * kTileWarps * 32) * 4;
+                    const int c = i / kTileDC, j = i % kTileDC;
+                    tmp[u] = (e0 + c < E && j < dn)
+                                 ? *reinterpret_cast<const float4 *>(W_g + static_cast<int64_t>(e0 + c) * d + dc + j)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < kPieces; ++u)
+                    reinterpret_cast<float4 *>(ws)[threadIdx.x + u * kTileWarps * 32] = tmp[u];
+            } else {
+                for (int i = threadIdx.x; i < kTileEC * kTileDC; i += blockDim.x) {
+                    const int c = i / kTileDC, j = i % kTileDC;
+                    ws[i] = (e0 + c < E && j < dn) ? W_g[static_cast<int64_t>(e0 + c) * d + dc + j] : 0.0f;
+                }
+            }
+            __syncthreads();
+            if (ntok > 0) {
+#pragma unroll 2
+                for (int j = lane * VEC; j < dn; j += 32 * VEC) {
+                    float xv[kTileTPW][VEC];
+#pragma unroll
+                    for (int a = 0; a < kTileTPW; ++a) {
+                        if (a < ntok) {
+                            XLoad<T, VEC>::load(x + (t0 + a) * static_cast<int64_t>(d) + dc + j, xv[a]);
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) xv[a][v] = 0.0f;
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < kTileEC; ++c) {
                         float w[VEC];
-                        load_w<VEC>(W_g + static_cast<int64_t>(e0 + c) * d + i, w);
+                        load_w<VEC>(ws + c * kTileDC + j, w);
 #pragma unroll
-                        for (int v = 0; v < VEC; ++v) acc[c] = fmaf(xv[v], w[v], acc[c]);
+                        for (int a = 0; a < kTileTPW; ++a)
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) acc[a][c] = fmaf(xv[a][v], w[v], acc[a][c]);
                     }
                 }
             }
         }
 #pragma unroll
-        for (int c = 0; c < EC; ++c) part[(warp * 32 + lane) * (EC + 1) + c] = acc[c];
-        __syncthreads();
-        if (warp == 0 && live) {
+        for (int a = 0; a < kTileTPW; ++a)
 #pragma unroll
-            for (int c = 0; c < EC; ++c) {
-                if (e0 + c < E) {
-                    float v = part[lane * (EC + 1) + c];
+            for (int c = 0; c < kTileEC; ++c) {
+                float v = acc[a][c];
 #pragma unroll
-                    for (int w = 1; w < kLaneWarps; ++w) v = __fadd_rn(v, part[(w * 32 + lane) * (EC + 1) + c]);
-                    if (b_g) v = __fadd_rn(v, b_g[e0 + c]);
-                    sc[lane * (E + 1) + e0 + c] = v;
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                acc[a][c] = v;
+            }
+        if (lane == 0) {
+#pragma unroll
+            for (int a = 0; a < kTileTPW; ++a)
+#pragma unroll
+                for (int c = 0; c < kTileEC; ++c)
+                    if (a < ntok && e0 + c < E) {
+                        float v = acc[a][c];
+                        if (b_g) v = __fadd_rn(v, b_g[e0 + c]);
+                        s_sc[(warp * kTileTPW + a) * E + e0 + c] = v;
+                    }
+        }
+    }
+    __syncwarp();
+    const bool use_noise = (noise != nullptr) && (sigma != 0.0f);
+    for (int a = 0; a < ntok; ++a) {
+        const int64_t t = t0 + a;
+        float *sc = s_sc + (warp * kTileTPW + a) * E;
+        for (int e = lane; e < E; e += 32) {
+            const float v = sc[e];
+            if (logits_out) logits_out[t * E + e] = v;
+            if (use_noise) sc[e] = add_noise(v, sigma, noise[t * E + e]);
+        }
+        __syncwarp();
+        float pv = 0.0f;
+        int pe = -1;
+        for (int j = 0; j < k; ++j) {
+            float bv = 0.0f;
+            int be = -1;
+            for (int e = lane; e < E; e += 32) {
+                const float v = sc[e];
+                if ((pe < 0 || ranks_before(pv, pe, v, e)) && (be < 0 || ranks_before(v, e, bv, be))) {
+                    bv = v;
+                    be = e;
                 }
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (oe >= 0 && (be < 0 || ranks_before(ov, oe, bv, be))) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            if (lane == 0) {
+                pick_v[j] = bv;
+                pick_e[j] = be;
+            }
+            pv = bv;
+            pe = be;
         }
-        __syncthreads();
-    }
-    if (warp != 0 || !live) return;
-
-    float *s = sc + lane * (E + 1);
-    const bool use_noise = (noise != nullptr) && (sigma != 0.0f);
-    for (int e = 0; e < E; ++e) {
-        if (logits_out) logits_out[t * E + e] = s[e];
-        if (use_noise) s[e] = add_noise(s[e], sigma, noise[t * E + e]);
-    }
-    // k picks in (score desc, index asc) order; softmax shifted by the first pick
-    float pv = 0.0f, m = 0.0f, sum = 0.0f;
-    int pe = -1;
-    for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int be = -1;
-        for (int e = 0; e < E; ++e) {
-            const float v = s[e];
-            if ((pe < 0 || ranks_before(pv, pe, v, e)) && (be < 0 || ranks_before(v, e, bv, be))) {
-                bv = v;
-                be = e;
+        __syncwarp();
+        if (lane == 0) {
+            const float m = pick_v[0];
+            float sum = 0.0f;
+            for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(pick_v[j], m)));
+            for (int j = 0; j < k; ++j) {
+                topk_idx[t * k + j] = pick_e[j];
+                gates[t * k + j] = __fdiv_rn(expf(__fsub_rn(pick_v[j], m)), sum);
             }
         }
-        if (j == 0) m = bv;
-        sum = __fadd_rn(sum, expf(__fsub_rn(bv, m)));
-        topk_idx[t * k + j] = be;
-        pv = bv;
-        pe = be;
-    }
-    for (int j = 0; j < k; ++j) {
-        const float v = s[topk_idx[t * k + j]];
-        gates[t * k + j] = __fdiv_rn(expf(__fsub_rn(v, m)), sum);
+        __syncwarp();
     }
 }
 
@@ -182,6 +248,8 @@ route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
                    int64_t N, int d, int E, int k, float *__restrict__ logits_out,
                    int32_t *__restrict__ topk_idx, float *__restrict__ gates,
                    uint32_t *__restrict__ status) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ float route_smem[];
     float *part = route_smem;          // [4 warps][kEC]
     float *sc = part + 4 * kEC;        // [E]
@@ -195,6 +263,7 @@ route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
         float acc[kEC];
 #pragma unroll
         for (int c = 0; c < kEC; ++c) acc[c] = 0.0f;
+#pragma unroll 4
         for (int i = threadIdx.x * VEC; i < d; i += 128 * VEC) {
             float xv[VEC];
             XLoad<T, VEC>::load(xr + i, xv);
@@ -280,20 +349,19 @@ cudaError_t launch_route_v(const void *x, const float *W_g, const float *b_g, co
     const T *xt = static_cast<const T *>(x);
     if (N <= kRouteBlockMaxN) {
         const size_t smem = sizeof(float) * (4 * kEC + E + 2 * static_cast<size_t>(k));
-        route_block_kernel<T, VEC><<<static_cast<unsigned>(N), 128, smem, s>>>(
-            xt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
-        return cudaGetLastError();
+        return launch_pdl(route_block_kernel<T, VEC>, dim3(static_cast<unsigned>(N)), dim3(128), smem, s, xt, W_g,
+                          b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
     }
-    const int64_t blocks = (N + 31) / 32;
-    if (E <= 8) {
-        const size_t smem = sizeof(float) * (kLaneWarps * 32 * (8 + 1) + 32 * (E + 1));
-        route_lanes_kernel<T, VEC, 8><<<static_cast<unsigned>(blocks), kLaneWarps * 32, smem, s>>>(
-            xt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
-    } else {
-        const size_t smem = sizeof(float) * (kLaneWarps * 32 * (16 + 1) + 32 * (E + 1));
-        route_lanes_kernel<T, VEC, 16><<<static_cast<unsigned>(blocks), kLaneWarps * 32, smem, s>>>(
-            xt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
+    const int64_t blocks = (N + kTileTok - 1) / kTileTok;
+    const size_t smem = sizeof(float) * (static_cast<size_t>(kTileEC) * kTileDC +
+                                         static_cast<size_t>(kTileTok) * E + static_cast<size_t>(kTileWarps) * 2 * k);
+    auto kern = route_tile_kernel<T, VEC>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
     }
+    return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kTileWarps * 32), smem, s, xt, W_g, b_g,
+                      noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
     return cudaGetLastError();
 }
 

@@ -17,12 +17,14 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libmoe.so")
 
 MOE_F32, MOE_BF16 = 0, 1
+ACT_RELU, ACT_GELU = 1, 2
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
 EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
-           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
-           "moe_forward", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
+           "moe_shard_workspace_size", "moe_shard_count", "moe_shard_base", "moe_shard_dispatch",
+           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_combine",
+           "moe_workspace_size", "moe_forward", "moe_forward_ex", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
 
 class MoeError(RuntimeError):
@@ -54,11 +56,18 @@ def load_library(path: str = LIB_PATH):
             "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
             "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
             "moe_dispatch_noalloc": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P]),
+            "moe_shard_workspace_size": (SZ, [I64, I, I]),
+            "moe_shard_count": (I, [P, I64, I, I, P, P, SZ, P]),
+            "moe_shard_base": (I, [P, I, I, I, I, P, P]),
+            "moe_shard_dispatch": (I, [P, P, I, I64, I, I, I, I64, P, P, P, P, P, P, P, SZ, P]),
             "moe_expert_ffn_workspace_size": (SZ, [I64, I, I, I, I]),
             "moe_expert_ffn": (I, [P, P, P, P, P, I, I64, I, I, I, P, P, SZ, P]),
+            "moe_expert_ffn_ex": (I, [P, P, P, P, P, I, I64, I, I, I, I, P, P, P, P, SZ, P]),
             "moe_combine": (I, [P, P, P, P, P, I, I64, I, I, P, P]),
             "moe_workspace_size": (SZ, [I64, I, I, I, I, D, I]),
             "moe_forward": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_forward_ex": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, I, P, P, P, P, P, P, P, P, P, SZ,
+                                   P]),
             "moe_forward_launches": (I, [I64, I, I, I, I, D, I]),
             "moe_check_status": (I, [P, P, ctypes.POINTER(U32)]),
             "moe_debug_wait_timeout": (I, [U32, P, SZ, P]),
@@ -184,8 +193,50 @@ def moe_dispatch_noalloc(topk_idx, x, E, cf, stream=None):
                 C=capacity(N, E, k, cf))
 
 
-def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=None, out=None):
-    """-> out_gathered [rows, d] (rows outside the kept ranges unspecified)."""
+def moe_shard_count(topk_idx, E, ws, stream=None):
+    """This shard's [k, E] int32 counts of j-th choices per expert (device).
+    `ws` (from shard_workspace) must then go, untouched, to moe_shard_dispatch."""
+    L = load_library()
+    N, k = topk_idx.shape
+    counts_je = torch.empty((k, E), dtype=torch.int32, device=topk_idx.device)
+    _check(L.moe_shard_count(_p(topk_idx), N, E, k, _p(counts_je), _p(ws), ws.numel(), _stream(stream)))
+    return counts_je
+
+
+def shard_workspace(N_local, E, k, device):
+    n = load_library().moe_shard_workspace_size(N_local, E, k)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def moe_shard_base(all_counts, rank, stream=None):
+    """all_counts [G, k, E] int32 (device, rank order) -> base [k, E] int32."""
+    L = load_library()
+    G, k, E = all_counts.shape
+    base = torch.empty((k, E), dtype=torch.int32, device=all_counts.device)
+    _check(L.moe_shard_base(_p(all_counts.contiguous()), G, rank, E, k, _p(base), _stream(stream)))
+    return base
+
+
+def moe_shard_dispatch(topk_idx, x, E, C, counts_je, base, ws, stream=None):
+    """-> dict(slot, counts, offsets, x_gathered, rows) for this shard."""
+    L = load_library()
+    N, d = x.shape
+    k = topk_idx.shape[1]
+    dev = x.device
+    rows = (N * k + 127) // 128 * 128
+    slot = torch.empty((N, k), dtype=torch.int32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    xg = torch.empty((rows, d), dtype=x.dtype, device=dev)
+    _check(L.moe_shard_dispatch(_p(topk_idx), _p(x), _dt(x), N, d, E, k, int(C), _p(counts_je), _p(base),
+                                _p(slot), _p(counts), _p(offsets), _p(xg), _p(ws), ws.numel(), _stream(stream)))
+    return dict(slot=slot, counts=counts, offsets=offsets, x_gathered=xg, rows=rows)
+
+
+def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=None, out=None, act=ACT_RELU,
+                   b_up=None, b_down=None):
+    """-> out_gathered [rows, d] (rows outside the kept ranges unspecified).
+    act/b_up/b_down select the nanoMoE expert variant (GELU, biases)."""
     L = load_library()
     for t, n in ((x_gathered, "x_gathered"), (offsets, "offsets"), (counts, "counts"), (W_up, "W_up"),
                  (W_down, "W_down")):
@@ -198,8 +249,11 @@ def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=No
         ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=x_gathered.device)
     if out is None:
         out = torch.empty((rows, d), dtype=x_gathered.dtype, device=x_gathered.device)
-    _check(L.moe_expert_ffn(_p(x_gathered), _p(offsets), _p(counts), _p(W_up), _p(W_down), dt, rows, d,
-                            d_ff, E, _p(out), _p(ws), ws.numel(), _stream(stream)))
+    for t, n in ((b_up, "b_up"), (b_down, "b_down")):
+        _cuda(t, n)
+    _check(L.moe_expert_ffn_ex(_p(x_gathered), _p(offsets), _p(counts), _p(W_up), _p(W_down), dt, rows, d,
+                               d_ff, E, int(act), _p(b_up), _p(b_down), _p(out), _p(ws), ws.numel(),
+                               _stream(stream)))
     return out
 
 
@@ -226,11 +280,12 @@ def forward_launches(N, d, E, d_ff, k, cf, dtype) -> int:
 
 
 def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=None, ws=None,
-                intermediates=False, stream=None):
-    """The whole layer.  -> y, or (y, dict of logits/topk_idx/gates/slot/counts)."""
+                intermediates=False, stream=None, act=ACT_RELU, b_up=None, b_down=None):
+    """The whole layer.  -> y, or (y, dict of logits/topk_idx/gates/slot/counts).
+    act/b_up/b_down select the nanoMoE expert variant (GELU, biases)."""
     L = load_library()
     for t, n in ((x, "x"), (W_g, "W_g"), (W_up, "W_up"), (W_down, "W_down"), (b_g, "b_g"),
-                 (noise, "noise")):
+                 (noise, "noise"), (b_up, "b_up"), (b_down, "b_down")):
         _cuda(t, n)
     N, d = x.shape
     E, d_ff, _ = W_up.shape
@@ -250,9 +305,10 @@ def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=
                      slot=torch.empty((N, k), dtype=torch.int32, device=dev),
                      counts=torch.empty(E, dtype=torch.int32, device=dev))
     g = (lambda n: _p(inter[n])) if inter else (lambda n: None)
-    _check(L.moe_forward(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, d_ff, k,
-                         _cf(cf), _p(W_up), _p(W_down), _p(y), g("logits"), g("topk_idx"), g("gates"),
-                         g("slot"), g("counts"), _p(ws), ws.numel(), _stream(stream)))
+    _check(L.moe_forward_ex(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, d_ff, k,
+                            _cf(cf), _p(W_up), _p(W_down), int(act), _p(b_up), _p(b_down), _p(y),
+                            g("logits"), g("topk_idx"), g("gates"), g("slot"), g("counts"), _p(ws),
+                            ws.numel(), _stream(stream)))
     return (y, inter) if intermediates else y
 
 
@@ -272,8 +328,10 @@ class MoELayer:
     """Weights resident on the device plus a reusable workspace; __call__ runs
     moe_forward on the current stream without allocating."""
 
-    def __init__(self, W_g, W_up, W_down, k, cf, b_g=None, sigma=0.0, max_tokens=None):
+    def __init__(self, W_g, W_up, W_down, k, cf, b_g=None, sigma=0.0, max_tokens=None, act=ACT_RELU,
+                 b_up=None, b_down=None):
         self.W_g, self.W_up, self.W_down, self.b_g = W_g, W_up, W_down, b_g
+        self.act, self.b_up, self.b_down = int(act), b_up, b_down
         self.k, self.cf, self.sigma = int(k), cf, float(sigma)
         self.E, self.d_ff, self.d = W_up.shape
         self._ws = None
@@ -295,7 +353,8 @@ class MoELayer:
         if self._ws is None or x.shape[0] != self._ws_tokens:
             self._reserve(x.shape[0], x.dtype)
         return moe_forward(x, self.W_g, self.W_up, self.W_down, self.k, self.cf, b_g=self.b_g,
-                           noise=noise, sigma=self.sigma, y=y, ws=self._ws, stream=stream)
+                           noise=noise, sigma=self.sigma, y=y, ws=self._ws, stream=stream, act=self.act,
+                           b_up=self.b_up, b_down=self.b_down)
 
 
 class GraphedForward:

@@ -79,11 +79,11 @@ def check_routing(case: Case, inter, logits_tol=None):
     wl, i = case.wl, case.inp
     lg = inter["logits"].cpu().numpy()
     ref_lg = oracle.router_logits(i.x, i.W_g, i.b_g)
-    # fp32 summation error bound for a depth-(d/4 + 16) accumulation of the
+    # fp32 summation error bound for a depth-(d/8 + 16) accumulation of the
     # products, plus one rounding of the result and the bias add
     absdot = np.abs(values(i.x)) @ np.abs(i.W_g.astype(np.float64)).T
     eps = 2.0 ** -24
-    bound = (wl.d / 4 + 16) * eps * absdot + 2 * eps * np.abs(ref_lg) + 1e-30
+    bound = (wl.d / 8 + 16) * eps * absdot + 2 * eps * np.abs(ref_lg) + 1e-30
     if logits_tol is not None:
         bound = np.maximum(bound, logits_tol)
     err = np.abs(lg.astype(np.float64) - ref_lg.astype(np.float64))

@@ -310,7 +310,61 @@ def check_all_dropped_is_zero(seed=9):
     np.testing.assert_allclose(out["y"][0], ref0, rtol=1e-12, atol=1e-12)
 
 
+def check_gelu_expert_variant(seed=12):
+    """nanoMoE slide 32 variant: GELU is x * Phi(x) with Phi the normal CDF
+    (scipy.stats.norm.cdf, a library routine), at printed-in-every-table points
+    and on random inputs; the biases are added after each projection."""
+    from scipy.stats import norm
+    z = np.array([0.0, 1.0, -1.0, 2.5, -3.0, 0.3], dtype=np.float32)
+    x = np.ones((1, 1), dtype=np.float32)
+    W_up = z.reshape(1, -1, 1)
+    W_down = np.ones((1, 1, z.size), dtype=np.float32)
+    h, o = oracle.expert_ffn_ex(x, W_up, W_down, 0, 0, act=oracle.ACT_GELU)
+    ref = z.astype(np.float64) * norm.cdf(z.astype(np.float64))
+    np.testing.assert_allclose(h, ref, rtol=1e-13, atol=1e-15)
+    assert h[0] == 0.0 and abs(h[1] - 0.8413447460685429) < 1e-14 and abs(h[2] + 0.15865525393145707) < 1e-14
+    rng = np.random.default_rng(seed)
+    E, d, d_ff = 2, 5, 7
+    x = rng.standard_normal((3, d)).astype(np.float32)
+    W_up = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    b_up = rng.standard_normal((E, d_ff)).astype(np.float32)
+    b_down = rng.standard_normal((E, d)).astype(np.float32)
+    x64, u64, w64 = (a.astype(np.float64) for a in (x, W_up, W_down))
+    for act in (oracle.ACT_RELU, oracle.ACT_GELU):
+        for t in range(3):
+            for e in range(E):
+                h, o = oracle.expert_ffn_ex(x, W_up, W_down, t, e, act=act, b_up=b_up, b_down=b_down)
+                zz = u64[e] @ x64[t] + b_up[e].astype(np.float64)
+                hh = np.maximum(zz, 0) if act == oracle.ACT_RELU else zz * norm.cdf(zz)
+                np.testing.assert_allclose(h, hh, rtol=1e-12, atol=1e-12)
+                np.testing.assert_allclose(o, w64[e] @ hh + b_down[e].astype(np.float64), rtol=1e-12, atol=1e-12)
+    # the plain layer is the variant with ReLU and no biases
+    h0, o0 = oracle.expert_ffn(x, W_up, W_down, 1, 1)
+    h1, o1 = oracle.expert_ffn_ex(x, W_up, W_down, 1, 1, act=oracle.ACT_RELU)
+    assert np.array_equal(h0, h1) and np.array_equal(o0, o1)
+
+
+def check_gelu_bias_layer(seed=13):
+    """E = 1, k = 1 with GELU and biases is the dense nanoMoE MLP."""
+    from scipy.stats import norm
+    rng = np.random.default_rng(seed)
+    N, d, d_ff = 6, 4, 10
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    W_g = rng.standard_normal((1, d)).astype(np.float32)
+    W_up = rng.standard_normal((1, d_ff, d)).astype(np.float32)
+    W_down = rng.standard_normal((1, d, d_ff)).astype(np.float32)
+    b_up = rng.standard_normal((1, d_ff)).astype(np.float32)
+    b_down = rng.standard_normal((1, d)).astype(np.float32)
+    out = oracle.forward(x, W_g, None, None, 0.0, 1, 1.0, W_up, W_down, act=oracle.ACT_GELU,
+                         b_up=b_up, b_down=b_down)
+    z = x.astype(np.float64) @ W_up[0].T.astype(np.float64) + b_up[0].astype(np.float64)
+    ref = (z * norm.cdf(z)) @ W_down[0].T.astype(np.float64) + b_down[0].astype(np.float64)
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+
+
 ALL_CHECKS = [check_m1, check_m2_slots, check_m2_combine, check_topk_bruteforce,
               check_gates_invariants, check_noise, check_capacity, check_slots_bruteforce,
               check_logits_vs_numpy, check_ffn_vs_numpy, check_dense_mixture,
-              check_single_expert_mlp, check_all_dropped_is_zero]
+              check_single_expert_mlp, check_all_dropped_is_zero, check_gelu_expert_variant,
+              check_gelu_bias_layer]

@@ -37,6 +37,11 @@ MUTANTS = {
                              "counts[e] = (int32_t)queue[e];"),
     "bias_dropped": ("s = s + b_g[e];", "s = s + 0.0f * b_g[e];"),
     "gate_not_applied": ("yt[i] += g * o[i];", "yt[i] += o[i];"),
+    "gelu_as_relu": ("if (act == 2)\n            h[f] = 0.5 * z * (1.0 + erf(z / sqrt(2.0)));",
+                     "if (act == 3)\n            h[f] = 0.5 * z * (1.0 + erf(z / sqrt(2.0)));"),
+    "gelu_unscaled_erf": ("erf(z / sqrt(2.0))", "erf(z)"),
+    "up_bias_dropped": ("z += (double)b_up[(size_t)e * d_ff + f];", "z += 0.0 * b_up[(size_t)e * d_ff + f];"),
+    "down_bias_dropped": ("acc += (double)b_down[(size_t)e * d + i];", "acc += 0.0 * b_down[(size_t)e * d + i];"),
     "softmax_not_shifted_sign": ("denom += exp((double)s[idx[j]] - top);",
                                  "denom += exp(top - (double)s[idx[j]]);"),
 }
@@ -62,7 +67,8 @@ def test_pins_catch_mutant(tmp_path, name):
     try:
         mutant = ctypes.CDLL(lib_path)
         for fn in ("oracle_router_logits", "oracle_route_from_logits", "oracle_capacity",
-                   "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine"):
+                   "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine",
+                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex"):
             getattr(mutant, fn).argtypes = getattr(saved, fn).argtypes
             getattr(mutant, fn).restype = getattr(saved, fn).restype
         O._lib = mutant
