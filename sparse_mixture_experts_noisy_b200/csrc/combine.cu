@@ -7,7 +7,8 @@
 // The dense [tokens, E*C] x [E*C, d] product of the slides is replaced by a
 // gather: for each token, threads own chunks of its output columns, read those
 // chunks of the token's k expert-output rows and accumulate g * row in fp32, in
-// choice order j = 0..k-1.  A block takes one token at a time.
+// choice order j = 0..k-1.  Small batches give a token to a whole block in
+// turn; large ones give each grid row one token, one chunk per thread.
 //
 // The expert outputs are either rows of dtype T (one partial) or `parts`
 // fp32 partial sums over K-splits of the down projection, which are added in
@@ -135,14 +136,71 @@ combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, 
     }
 }
 
+// Large batches: grid rows are tokens, grid columns are 128-chunk pieces of
+// the token's columns; one chunk per thread and no block-wide barrier, so many
+// tokens' loads are in flight at once.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(128)
+combine_flat_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, int nparts,
+                    int64_t part_stride, const int32_t *__restrict__ slot,
+                    const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
+                    const float *__restrict__ gates, int64_t N, int d, int k, int E,
+                    T *__restrict__ y, const float *__restrict__ b_down) {
+    pdl_trigger();
+    pdl_wait();
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) * VEC;
+    if (c >= d) return;
+    for (int64_t t = blockIdx.y; t < N; t += gridDim.y) {
+        float acc[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int32_t sl = slot[t * k + j];
+            const int32_t e = topk_idx[t * k + j];
+            if (sl < 0 || e < 0 || e >= E) continue;
+            const int64_t r = static_cast<int64_t>(offsets[e]) + sl;
+            const float gj = gates[t * k + j];
+            float o[VEC];
+            if (nparts == 0) {
+                Vec<T, VEC>::load(out_rows + r * d + c, o);
+            } else {
+                load_f32<VEC>(parts + r * d + c, o);
+#pragma unroll 4
+                for (int p = 1; p < nparts; ++p) {
+                    float q[VEC];
+                    load_f32<VEC>(parts + p * part_stride + r * d + c, q);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) o[v] += q[v];
+                }
+                if (b_down != nullptr) {
+                    float bq[VEC];
+                    load_f32<VEC>(b_down + static_cast<int64_t>(e) * d + c, bq);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) o[v] += bq[v];
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj, o[v], acc[v]);
+        }
+        Vec<T, VEC>::store(y + t * d + c, acc);
+    }
+}
+
 template <typename T, int VEC>
 cudaError_t launch_combine_t(const void *out_rows, const float *parts, int nparts,
                              int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
                              const int32_t *offsets, const float *gates, int64_t N, int d, int k,
                              int E, void *y, cudaStream_t s, const float *b_down) {
+    const int chunks = d / VEC;
+    if (N >= 2048) {
+        const unsigned gx = static_cast<unsigned>((chunks + 127) / 128);
+        const unsigned gy = static_cast<unsigned>(N < 65535 ? N : 65535);
+        return launch_pdl(combine_flat_kernel<T, VEC>, dim3(gx, gy), dim3(128), 0, s,
+                          static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets,
+                          gates, N, d, k, E, static_cast<T *>(y), b_down);
+    }
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int chunks = d / VEC;
     const int threads = chunks >= 256 ? 256 : (chunks >= 128 ? 128 : (chunks >= 64 ? 64 : 32));
     int64_t blocks = N;
     if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;

@@ -32,8 +32,8 @@
 // frees its tensor memory and exits.
 #include "common.cuh"
 #include "internal.h"
+#include "tmap.h"
 
-#include <cudaTypedefs.h>
 #include <cstdlib>
 
 namespace moe {
@@ -42,6 +42,7 @@ namespace {
 
 constexpr int kBM = 128;       // MMA M
 constexpr int kBK = 64;        // K elements per stage (128 bytes of bf16 = one swizzle row)
+static_assert(kBK == kTmapBoxK, "tensor-map box K");
 constexpr int kThreads = 192;
 
 // Epilogues: bf16 out with the optional bias (down projection), bf16 out with
@@ -655,54 +656,14 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *p = nullptr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// bf16 [rows, K] K-major, box = 64 (K) x box_rows, 128-byte swizzle.
-bool make_map_2d(CUtensorMap *m, const void *base, int64_t rows, int K, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// bf16 [E, Nw, K] K-major, box = 64 (K) x box_rows x 1, 128-byte swizzle.
-bool make_map_3d(CUtensorMap *m, const void *base, int E, int Nw, int K, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(Nw),
-                          static_cast<cuuint64_t>(E)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(K) * 2 * Nw};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows), 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int BN, bool SWAP, int EPI, int STAGES>
 cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
                       const int32_t *offsets, const int32_t *counts, int splits, void *out,
                       int64_t ldo, int64_t split_stride, uint32_t *status, uint64_t timeout_ns,
                       int grid, cudaStream_t s, const float *bias = nullptr, int act = 1) {
     CUtensorMap tm_tok, tm_w;
-    if (!make_map_2d(&tm_tok, tok, tok_rows, K, SWAP ? BN : kBM)) return cudaErrorInvalidValue;
-    if (!make_map_3d(&tm_w, W, E, Nw, K, SWAP ? kBM : BN)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tm_tok, tok, tok_rows, K, SWAP ? BN : kBM)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_3d(&tm_w, W, E, Nw, K, SWAP ? kBM : BN)) return cudaErrorInvalidValue;
     constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024;
     auto kern = tc_gemm_kernel<BN, SWAP, EPI, STAGES>;
     static bool attr_set = false;
@@ -721,8 +682,8 @@ cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, 
                        uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
                        const float *bias = nullptr, int act = 1) {
     CUtensorMap tm_tok, tm_w;
-    if (!make_map_2d(&tm_tok, tok, tok_rows, K, 128)) return cudaErrorInvalidValue;
-    if (!make_map_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tm_tok, tok, tok_rows, K, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
     constexpr int smem = STAGES * 2 * 128 * kBK * 2 + 1024;
     auto kern = tc2_gemm_kernel<EPI, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

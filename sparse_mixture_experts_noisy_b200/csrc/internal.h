@@ -34,6 +34,14 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
                          float *logits_out, int32_t *topk_idx, float *gates, uint32_t *status,
                          cudaStream_t s);
 
+// Tensor-core router for bf16 tokens (route_tc.cu): same results contract as
+// launch_route (logits within fp32 accumulation error of the exact dot
+// products; KeepTopK and softmax identical).  status nullable.
+bool route_tc_eligible(const void *x, const float *W_g, int64_t N, int d, int E);
+cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, const float *noise, float sigma,
+                            int64_t N, int d, int E, int k, float *logits_out, int32_t *topk_idx, float *gates,
+                            uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
+
 // Dispatch (dispatch.cu).
 int64_t dispatch_blocks(int64_t N);
 bool dispatch_single_block(int64_t N, int E, int k);

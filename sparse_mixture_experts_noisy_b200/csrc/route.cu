@@ -5,12 +5,14 @@
 // "nanoMoEの深層解剖" slides 11-13 (router in fp32 with autocast disabled, topk,
 // -inf scatter, softmax).
 //
-// The dot products run on CUDA cores in fp32 (fmaf).  Two launch shapes:
-// large batches give 4 tokens to each warp with W_g staged in shared memory,
-// small batches give one token to a whole block so that even 64 tokens spread
-// over the GPU.  The bias
-// and the noise are added with explicit round-to-nearest adds and multiplies,
-// so the compiler cannot fuse the noise step into one rounding.
+// bf16 tokens with d a multiple of 8 and at most 160 experts route on the
+// tensor cores (route_tc.cu).  Everything else runs here, on CUDA cores in
+// fp32 (fmaf), in one of two launch shapes: large batches give 4 tokens to
+// each warp with W_g staged in shared memory, small batches give one token to
+// a whole block.  Both sum every dot product in the same order, so the choice
+// between them never changes a result.  The bias and the noise are added with
+// explicit round-to-nearest adds and multiplies, so the compiler cannot fuse
+// the noise step into one rounding.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,6 +22,7 @@ namespace {
 
 constexpr int kEC = 8;                  // experts per accumulation pass (small batches)
 constexpr int64_t kRouteBlockMaxN = 1024; // up to this many tokens: one block per token
+constexpr uint64_t kRouteWaitTimeoutNs = 1000000000ull;  // tensor-core router: 1 s per wait
 
 template <typename T, int VEC>
 struct XLoad;
@@ -75,7 +78,7 @@ __device__ __forceinline__ float add_noise(float s, float sigma, float eps) {
 }
 
 // ------------------------------------------------------------------ large batches
-// A block of 8 warps owns 32 tokens, 4 per warp.  For each 512-wide chunk of
+// A block of 8 warps owns 32 tokens, 4 per warp.  For each 1024-wide chunk of
 // d the block stages W_g[e0 .. e0+8)[chunk] in shared memory; the lanes of a
 // warp read 16-byte pieces of their 4 tokens' rows (consecutive lanes,
 // consecutive bytes) and keep 4 tokens x 8 experts of fp32 partial sums, which
@@ -84,7 +87,7 @@ __device__ __forceinline__ float add_noise(float s, float sigma, float eps) {
 constexpr int kTileWarps = 8;
 constexpr int kTileTPW = 4;                    // tokens per warp
 constexpr int kTileTok = kTileWarps * kTileTPW;
-constexpr int kTileDC = 512;                   // d chunk staged per pass
+constexpr int kTileDC = 1024;                  // d chunk staged per pass
 constexpr int kTileEC = 8;                     // experts per pass
 
 template <typename T, int VEC>
@@ -139,7 +142,7 @@ route_tile_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
             }
             __syncthreads();
             if (ntok > 0) {
-#pragma unroll 2
+#pragma unroll 1
                 for (int j = lane * VEC; j < dn; j += 32 * VEC) {
                     float xv[kTileTPW][VEC];
 #pragma unroll
@@ -238,9 +241,13 @@ route_tile_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
 }
 
 // ------------------------------------------------------------------ small batches
-// One token per block: the 128 threads split d, each keeps 8 experts' partial
-// sums, the block adds them (shuffles, then the 4 warps in order), and warp 0
-// runs k rounds of a warp-wide (score desc, index asc) arg-max and the softmax.
+// One token per block, so that even a few tokens spread over the GPU.  Warp w
+// takes experts w, w+4, w+8, ... (kEC of them per pass) and sums each dot
+// product exactly as the large-batch kernel does: lane l runs one fmaf chain
+// over the VEC-wide pieces l, l+32, l+64, ... of d, then the warp adds the
+// lanes with the same xor-shuffle tree.  So a token gets the same logits, bit
+// for bit, whatever the batch size.  Warp 0 then runs k rounds of a warp-wide
+// (score desc, index asc) arg-max and the softmax.
 template <typename T, int VEC>
 __global__ void __launch_bounds__(128)
 route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
@@ -251,27 +258,27 @@ route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
     pdl_trigger();
     pdl_wait();
     extern __shared__ float route_smem[];
-    float *part = route_smem;          // [4 warps][kEC]
-    float *sc = part + 4 * kEC;        // [E]
+    float *sc = route_smem;            // [E]
     float *pick_v = sc + E;            // [k]
     int *pick_e = reinterpret_cast<int *>(pick_v + k);  // [k]
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = blockIdx.x;
     const T *xr = x + t * static_cast<int64_t>(d);
-    for (int e0 = 0; e0 < E; e0 += kEC) {
+    for (int g0 = warp; g0 < E; g0 += 4 * kEC) {  // experts g0 + 4c, c < kEC
         float acc[kEC];
 #pragma unroll
         for (int c = 0; c < kEC; ++c) acc[c] = 0.0f;
-#pragma unroll 4
-        for (int i = threadIdx.x * VEC; i < d; i += 128 * VEC) {
+#pragma unroll 1
+        for (int j = lane * VEC; j < d; j += 32 * VEC) {
             float xv[VEC];
-            XLoad<T, VEC>::load(xr + i, xv);
+            XLoad<T, VEC>::load(xr + j, xv);
 #pragma unroll
             for (int c = 0; c < kEC; ++c) {
-                if (e0 + c < E) {
+                const int e = g0 + 4 * c;
+                if (e < E) {
                     float w[VEC];
-                    load_w<VEC>(W_g + static_cast<int64_t>(e0 + c) * d + i, w);
+                    load_w<VEC>(W_g + static_cast<int64_t>(e) * d + j, w);
 #pragma unroll
                     for (int v = 0; v < VEC; ++v) acc[c] = fmaf(xv[v], w[v], acc[c]);
                 }
@@ -282,18 +289,11 @@ route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
             float v = acc[c];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) part[warp * kEC + c] = v;
+            const int e = g0 + 4 * c;
+            if (lane == 0 && e < E) sc[e] = b_g ? __fadd_rn(v, b_g[e]) : v;
         }
-        __syncthreads();
-        if (threadIdx.x < kEC && e0 + threadIdx.x < E) {
-            const int c = threadIdx.x;
-            float v = part[c];
-            for (int w = 1; w < 4; ++w) v = __fadd_rn(v, part[w * kEC + c]);
-            if (b_g) v = __fadd_rn(v, b_g[e0 + c]);
-            sc[e0 + c] = v;
-        }
-        __syncthreads();
     }
+    __syncthreads();
     if (warp != 0) return;
     const bool use_noise = (noise != nullptr) && (sigma != 0.0f);
     for (int e = lane; e < E; e += 32) {
@@ -348,7 +348,7 @@ cudaError_t launch_route_v(const void *x, const float *W_g, const float *b_g, co
                            int32_t *topk_idx, float *gates, uint32_t *status, cudaStream_t s) {
     const T *xt = static_cast<const T *>(x);
     if (N <= kRouteBlockMaxN) {
-        const size_t smem = sizeof(float) * (4 * kEC + E + 2 * static_cast<size_t>(k));
+        const size_t smem = sizeof(float) * (E + 2 * static_cast<size_t>(k));
         return launch_pdl(route_block_kernel<T, VEC>, dim3(static_cast<unsigned>(N)), dim3(128), smem, s, xt, W_g,
                           b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status);
     }
@@ -373,6 +373,9 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
                          cudaStream_t s) {
     if (N == 0) return status ? cudaMemsetAsync(status, 0, sizeof(uint32_t), s) : cudaSuccess;
     const uintptr_t ax = reinterpret_cast<uintptr_t>(x), aw = reinterpret_cast<uintptr_t>(W_g);
+    if (dt == 1 && route_tc_eligible(x, W_g, N, d, E))
+        return launch_route_tc(x, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status,
+                               kRouteWaitTimeoutNs, s);
     if (dt == 1) {
         if (d % 8 == 0 && ax % 16 == 0 && aw % 16 == 0)
             return launch_route_v<__nv_bfloat16, 8>(x, W_g, b_g, noise, sigma, N, d, E, k,
