@@ -83,7 +83,7 @@ size_t ffn_ws_bytes(int64_t rows, int d, int E, int d_ff, moe_dtype dt) {
 }
 
 struct FwdLayout {
-    size_t status, topk, gates, slot, counts, offsets, dws, xg, og, ffn, total;
+    size_t status, topk, gates, slot, counts, offsets, dws, w3, xg, og, ffn, total;
 };
 
 FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows, moe_dtype dt) {
@@ -98,6 +98,7 @@ FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows,
     L.counts = o; o += align_up(static_cast<size_t>(E) * 4, 256);
     L.offsets = o; o += align_up(static_cast<size_t>(E + 1) * 4, 256);
     L.dws = o; o += moe::dispatch_ws_bytes(N, E, k);
+    L.w3 = o; o += (dt == MOE_BF16) ? moe::route_tc_w3_bytes(d, E) : 0;  // pre-split router weights
     L.xg = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
     L.og = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
     L.ffn = o; o += ffn_ws_bytes(rows, d, E, d_ff, dt);
@@ -454,8 +455,9 @@ moe_status moe_forward_ex(const void *x, moe_dtype dt, const float *W_g, const f
     void *xg = w + L.xg;
     void *og = w + L.og;
 
+    void *w3 = (L.xg > L.w3) ? static_cast<void *>(w + L.w3) : nullptr;
     cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
-                                      logits_out, topk, gates, status, s);
+                                      logits_out, topk, gates, status, s, w3);
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
     if (N == 0) {
         if (counts_out) {
@@ -497,8 +499,9 @@ int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, mo
         const int64_t rows = rows_for(N, E, k, moe_capacity(N, E, k, cf));
         ffn = moe::tc_ffn_launches(moe::plan_tc_ffn(rows, d, d_ff, E, num_sms_current()), true);
     }
-    // router + dispatch passes + expert FFN + combine
-    return 1 + moe::dispatch_launches(N, E, k) + ffn + 1;
+    // router (+ its weight split) + dispatch passes + expert FFN + combine
+    const bool w3 = dt == MOE_BF16 && moe::route_tc_w3_bytes(d, E) > 0;
+    return moe::route_launches(dt == MOE_BF16 ? 1 : 0, N, d, E, k, w3) + moe::dispatch_launches(N, E, k) + ffn + 1;
 }
 
 moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {

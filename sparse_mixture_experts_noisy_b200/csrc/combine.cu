@@ -8,7 +8,7 @@
 // gather: for each token, threads own chunks of its output columns, read those
 // chunks of the token's k expert-output rows and accumulate g * row in fp32, in
 // choice order j = 0..k-1.  Small batches give a token to a whole block in
-// turn; large ones give each grid row one token, one chunk per thread.
+// turn; large ones give each thread one chunk of one token.
 //
 // The expert outputs are either rows of dtype T (one partial) or `parts`
 // fp32 partial sums over K-splits of the down projection, which are added in
@@ -24,6 +24,17 @@ template <typename T, int VEC>
 struct Vec;
 template <>
 struct Vec<__nv_bfloat16, 8> {
+    using Raw = uint4;
+    static __device__ __forceinline__ Raw load_raw(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint4 *>(p); }
+    static __device__ __forceinline__ void widen(const Raw &u, float (&v)[8]) {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(h[i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    }
     static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
         uint4 u = *reinterpret_cast<const uint4 *>(p);
         const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -44,6 +55,11 @@ struct Vec<__nv_bfloat16, 8> {
 };
 template <>
 struct Vec<float, 4> {
+    using Raw = float4;
+    static __device__ __forceinline__ Raw load_raw(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+    static __device__ __forceinline__ void widen(const Raw &u, float (&v)[4]) {
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    }
     static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
         float4 u = *reinterpret_cast<const float4 *>(p);
         v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
@@ -54,6 +70,9 @@ struct Vec<float, 4> {
 };
 template <typename T>
 struct Vec<T, 1> {
+    using Raw = T;
+    static __device__ __forceinline__ Raw load_raw(const T *p) { return *p; }
+    static __device__ __forceinline__ void widen(const Raw &u, float (&v)[1]) { v[0] = to_f32<T>(u); }
     static __device__ __forceinline__ void load(const T *p, float (&v)[1]) { v[0] = to_f32<T>(*p); }
     static __device__ __forceinline__ void store(T *p, const float (&v)[1]) { *p = from_f32<T>(v[0]); }
 };
@@ -136,54 +155,62 @@ combine_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, 
     }
 }
 
-// Large batches: grid rows are tokens, grid columns are 128-chunk pieces of
-// the token's columns; one chunk per thread and no block-wide barrier, so many
-// tokens' loads are in flight at once.
+// Large batches: each thread owns one VEC-wide chunk of one token's output
+// (blocks of 128 chunks; a token spans ceil(d / VEC / 128) blocks).  The
+// thread fetches the (slot, expert, gate) of up to kCombineGroup choices at
+// once, then their row offsets, then their data, so a token costs three
+// dependent memory round trips per group of choices rather than three per
+// choice; the adds still run in choice order j = 0..k-1, the same arithmetic
+// per element as the block kernel above.  Rows are dtype (nparts == 0).
+constexpr int kCombineGroup = 6;
+
 template <typename T, int VEC>
-__global__ void __launch_bounds__(128)
-combine_flat_kernel(const T *__restrict__ out_rows, const float *__restrict__ parts, int nparts,
-                    int64_t part_stride, const int32_t *__restrict__ slot,
-                    const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
-                    const float *__restrict__ gates, int64_t N, int d, int k, int E,
-                    T *__restrict__ y, const float *__restrict__ b_down) {
+__global__ void __launch_bounds__(128, 6)
+combine_token_kernel(const T *__restrict__ out_rows, const int32_t *__restrict__ slot,
+                     const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
+                     const float *__restrict__ gates, int64_t N, int d, int k, int E, int blocks_per_token,
+                     T *__restrict__ y) {
     pdl_trigger();
     pdl_wait();
-    const int c = (blockIdx.x * blockDim.x + threadIdx.x) * VEC;
-    if (c >= d) return;
-    for (int64_t t = blockIdx.y; t < N; t += gridDim.y) {
-        float acc[VEC];
+    const int64_t t = blockIdx.x / blocks_per_token;
+    const int c = ((blockIdx.x % blocks_per_token) * 128 + threadIdx.x) * VEC;
+    if (t >= N || c >= d) return;
+    float acc[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int32_t sl = slot[t * k + j];
-            const int32_t e = topk_idx[t * k + j];
-            if (sl < 0 || e < 0 || e >= E) continue;
-            const int64_t r = static_cast<int64_t>(offsets[e]) + sl;
-            const float gj = gates[t * k + j];
-            float o[VEC];
-            if (nparts == 0) {
-                Vec<T, VEC>::load(out_rows + r * d + c, o);
-            } else {
-                load_f32<VEC>(parts + r * d + c, o);
-#pragma unroll 4
-                for (int p = 1; p < nparts; ++p) {
-                    float q[VEC];
-                    load_f32<VEC>(parts + p * part_stride + r * d + c, q);
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+    for (int j0 = 0; j0 < k; j0 += kCombineGroup) {
+        int32_t sl[kCombineGroup], ex[kCombineGroup];
+        float g[kCombineGroup];
 #pragma unroll
-                    for (int v = 0; v < VEC; ++v) o[v] += q[v];
-                }
-                if (b_down != nullptr) {
-                    float bq[VEC];
-                    load_f32<VEC>(b_down + static_cast<int64_t>(e) * d + c, bq);
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) o[v] += bq[v];
-                }
+        for (int i = 0; i < kCombineGroup; ++i) {
+            const int j = j0 + i;
+            sl[i] = -1;
+            if (j < k) {
+                sl[i] = slot[t * k + j];
+                ex[i] = topk_idx[t * k + j];
+                g[i] = gates[t * k + j];
             }
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj, o[v], acc[v]);
         }
-        Vec<T, VEC>::store(y + t * d + c, acc);
+        int32_t r[kCombineGroup];
+#pragma unroll
+        for (int i = 0; i < kCombineGroup; ++i) {
+            const bool ok = sl[i] >= 0 && ex[i] >= 0 && ex[i] < E;
+            r[i] = ok ? offsets[ex[i]] + sl[i] : -1;
+        }
+        typename Vec<T, VEC>::Raw raw[kCombineGroup];
+#pragma unroll
+        for (int i = 0; i < kCombineGroup; ++i)
+            if (r[i] >= 0) raw[i] = Vec<T, VEC>::load_raw(out_rows + static_cast<int64_t>(r[i]) * d + c);
+#pragma unroll
+        for (int i = 0; i < kCombineGroup; ++i)
+            if (r[i] >= 0) {
+                float o[VEC];
+                Vec<T, VEC>::widen(raw[i], o);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[v] = fmaf(g[i], o[v], acc[v]);
+            }
     }
+    Vec<T, VEC>::store(y + t * d + c, acc);
 }
 
 template <typename T, int VEC>
@@ -192,15 +219,14 @@ cudaError_t launch_combine_t(const void *out_rows, const float *parts, int npart
                              const int32_t *offsets, const float *gates, int64_t N, int d, int k,
                              int E, void *y, cudaStream_t s, const float *b_down) {
     const int chunks = d / VEC;
-    if (N >= 2048) {
-        const unsigned gx = static_cast<unsigned>((chunks + 127) / 128);
-        const unsigned gy = static_cast<unsigned>(N < 65535 ? N : 65535);
-        return launch_pdl(combine_flat_kernel<T, VEC>, dim3(gx, gy), dim3(128), 0, s,
-                          static_cast<const T *>(out_rows), parts, nparts, part_stride, slot, topk_idx, offsets,
-                          gates, N, d, k, E, static_cast<T *>(y), b_down);
-    }
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int bpt = (chunks + 127) / 128;
+    if (N >= 2048 && nparts == 0 && N * bpt <= INT32_MAX) {
+        return launch_pdl(combine_token_kernel<T, VEC>, dim3(static_cast<unsigned>(N * bpt)), dim3(128), 0, s,
+                          static_cast<const T *>(out_rows), slot, topk_idx, offsets, gates, N, d, k, E, bpt,
+                          static_cast<T *>(y));
+    }
     const int threads = chunks >= 256 ? 256 : (chunks >= 128 ? 128 : (chunks >= 64 ? 64 : 32));
     int64_t blocks = N;
     if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;

@@ -323,6 +323,48 @@ gather_kernel(const U *__restrict__ x, int64_t units_per_row, const int32_t *__r
     }
 }
 
+// Large batches: one warp per token (grid-stride).  The warp reads the
+// token's row once, kGatherUnroll 16-byte pieces per lane in flight, and
+// writes it to each kept destination row; lanes j < k look the rows up.
+constexpr int kGatherUnroll = 8;
+
+__global__ void __launch_bounds__(256)
+gather_warp_kernel(const uint4 *__restrict__ x, int units, const int32_t *__restrict__ topk_idx,
+                   const int32_t *__restrict__ slot, const int32_t *__restrict__ offsets, int64_t N, int k,
+                   uint4 *__restrict__ xg) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t t = w0; t < N; t += nw) {
+        int32_t dest = -1;  // lane j < k: gathered row of choice j, or -1 if dropped
+        if (lane < k) {
+            const int32_t sl = slot[t * k + lane];
+            if (sl >= 0) dest = offsets[topk_idx[t * k + lane]] + sl;
+        }
+        const uint4 *xr = x + t * units;
+        for (int c0 = 0; c0 < units; c0 += 32 * kGatherUnroll) {
+            uint4 v[kGatherUnroll];
+#pragma unroll
+            for (int u = 0; u < kGatherUnroll; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < units) v[u] = xr[c];
+            }
+            for (int j = 0; j < k; ++j) {
+                const int32_t dj = __shfl_sync(0xffffffffu, dest, j);
+                if (dj < 0) continue;
+                uint4 *dr = xg + static_cast<int64_t>(dj) * units;
+#pragma unroll
+                for (int u = 0; u < kGatherUnroll; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < units) dr[c] = v[u];
+                }
+            }
+        }
+    }
+}
+
 }  // namespace
 
 int64_t dispatch_blocks(int64_t N) { return (N + kDispatchTB - 1) / kDispatchTB; }
@@ -428,6 +470,13 @@ cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const in
     const int64_t total = Nk * units;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (vec16 && N >= 2048 && k <= 32 && units <= INT32_MAX) {
+        int64_t blocks = (N + 7) / 8;  // 8 warps per block, one token per warp and pass
+        if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+        return launch_pdl(gather_warp_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                          static_cast<const uint4 *>(x), static_cast<int>(units), topk_idx, slot, offsets, N, k,
+                          static_cast<uint4 *>(x_gathered));
+    }
     int64_t blocks = (total + 255) / 256;
     if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
     if (blocks < 1) blocks = 1;

@@ -28,19 +28,28 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-// Router (route.cu).  status (nullable) is zeroed by the first block.
+// Router (route.cu).  status (nullable) is zeroed by the first block.  w3
+// (nullable): route_tc_w3_bytes(d, E) of scratch for the tensor-core router.
 cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b_g,
                          const float *noise, float sigma, int64_t N, int d, int E, int k,
                          float *logits_out, int32_t *topk_idx, float *gates, uint32_t *status,
-                         cudaStream_t s);
+                         cudaStream_t s, void *w3 = nullptr);
+// Kernels launch_route issues for 16-byte-aligned x and W_g (1, or 2 with w3
+// on the tensor-core path).
+int route_launches(int dt, int64_t N, int d, int E, int k, bool with_w3);
 
 // Tensor-core router for bf16 tokens (route_tc.cu): same results contract as
 // launch_route (logits within fp32 accumulation error of the exact dot
-// products; KeepTopK and softmax identical).  status nullable.
-bool route_tc_eligible(const void *x, const float *W_g, int64_t N, int d, int E);
+// products; KeepTopK and softmax identical).  status nullable.  w3 (nullable,
+// route_tc_w3_bytes) is scratch for the pre-split router weights: with it the
+// call launches a split pass first and the router reads the parts by TMA;
+// without it the router splits in-kernel.  Same results either way.
+bool route_tc_shape_ok(int64_t N, int d, int E, int k);  // bf16 tokens of this shape can use it
+bool route_tc_eligible(const void *x, const float *W_g, int64_t N, int d, int E, int k);
+size_t route_tc_w3_bytes(int d, int E);
 cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, const float *noise, float sigma,
                             int64_t N, int d, int E, int k, float *logits_out, int32_t *topk_idx, float *gates,
-                            uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
+                            uint32_t *status, uint64_t timeout_ns, void *w3, cudaStream_t s);
 
 // Dispatch (dispatch.cu).
 int64_t dispatch_blocks(int64_t N);

@@ -370,12 +370,12 @@ cudaError_t launch_route_v(const void *x, const float *W_g, const float *b_g, co
 cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b_g,
                          const float *noise, float sigma, int64_t N, int d, int E, int k,
                          float *logits_out, int32_t *topk_idx, float *gates, uint32_t *status,
-                         cudaStream_t s) {
+                         cudaStream_t s, void *w3) {
     if (N == 0) return status ? cudaMemsetAsync(status, 0, sizeof(uint32_t), s) : cudaSuccess;
     const uintptr_t ax = reinterpret_cast<uintptr_t>(x), aw = reinterpret_cast<uintptr_t>(W_g);
-    if (dt == 1 && route_tc_eligible(x, W_g, N, d, E))
+    if (dt == 1 && route_tc_eligible(x, W_g, N, d, E, k))
         return launch_route_tc(x, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status,
-                               kRouteWaitTimeoutNs, s);
+                               kRouteWaitTimeoutNs, w3, s);
     if (dt == 1) {
         if (d % 8 == 0 && ax % 16 == 0 && aw % 16 == 0)
             return launch_route_v<__nv_bfloat16, 8>(x, W_g, b_g, noise, sigma, N, d, E, k,
@@ -388,6 +388,11 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
                                         topk_idx, gates, status, s);
     return launch_route_v<float, 1>(x, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx,
                                     gates, status, s);
+}
+
+int route_launches(int dt, int64_t N, int d, int E, int k, bool with_w3) {
+    if (N == 0) return 0;
+    return (dt == 1 && route_tc_shape_ok(N, d, E, k) && with_w3) ? 2 : 1;
 }
 
 }  // namespace moe

@@ -1,5 +1,5 @@
 // Router on the fifth-generation tensor cores, for bf16 tokens: logits, noise,
-// KeepTopK and softmax over the kept scores in one kernel.
+// KeepTopK and softmax over the kept scores.
 //
 // "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター" STEP 2 (s_raw = W_g x),
 // STEP 4 (s = s_raw + eps), STEP 5 (-inf outside the top k), STEP 6 (softmax);
@@ -12,24 +12,32 @@
 // fp32 and the three 8-bit significands hold all 24 bits of w, so the sum is
 // w itself.  A bf16 token value times a bf16 part is exact in fp32 (16
 // significant bits), so every product the MMA forms is the exact fp32 product
-// x*w split in three; only the accumulation rounds, in fp32, as a CUDA-core
-// dot product would.  The three part-sums are added in the order hi, mid, lo.
+// x*w split in three; only the accumulation rounds, in fp32 (tensor memory).
+// The three part-sums are added in the order hi, mid, lo.
 //
 // Tile: 128 tokens (MMA M) x all experts.  B is the 3*E_pad rows
-// [w_hi of experts 0..E_pad-1; w_mid ...; w_lo ...] of one 64-wide K block,
-// written by the CTA's own threads into the 128-byte-swizzled K-major layout
-// the MMA reads; x arrives by TMA.  Accumulators: 3*E_pad fp32 columns of
-// tensor memory (column c = row c of B).
+// [w_hi of experts 0..E_pad-1; w_mid ...; w_lo ...] of one 64-wide K block in
+// the 128-byte-swizzled K-major layout the MMA reads.  Accumulators: 3*E_pad
+// fp32 columns of tensor memory (column c = row c of B).  B comes one of two
+// ways:
+//   - pre-split: a first small kernel writes the parts of all of W_g, once per
+//     call, to a [3*E_pad, d] bf16 scratch, and TMA loads B beside the x tile
+//     (the fused forward, which has a workspace);
+//   - in-kernel: TMA loads the fp32 W_g tile beside the x tile and four warps
+//     split it into the B slot (moe_route, which has none).
+// Both give the same B bits, so the same logits.
 //
-// Warp roles (192 threads): warp 0 lane 0 issues the x TMA loads into a
-// STAGES-deep ring; warp 1 owns the tensor memory and its lane 0 issues the
-// MMAs; warps 2-5 split W_g into the ring's B slots, then run the epilogue
-// (warp w reads TMEM lanes 32*(w%4)..+31, one token per thread): add the
-// three parts and the bias, write the logits (coalesced, through shared
-// memory), add the noise, pick the k best (score descending, lower expert
-// index first on ties) and form the softmax.  Every wait is bounded; on expiry
-// the kernel records ST_TIMEOUT, lets copies and MMAs in flight land, writes
-// expert -1 and gate 0 for its tokens, frees its tensor memory and exits.
+// The K range is cut into S pieces (S depends on d only); each piece is summed
+// from zero and the pieces are added in order, so a token's logits do not
+// depend on the batch size, on where the token sits, or on which of the two
+// kernel forms below ran:
+//   - clustered (few tiles): the S CTAs of a cluster each sum one piece of one
+//     tile and exchange the sums through distributed shared memory;
+//   - persistent (many tiles): one CTA per SM walks whole tiles, each piece in
+//     its own tensor-memory buffer (two, so MMAs and drains overlap).
+// Every wait is bounded; on expiry the kernel records ST_TIMEOUT, lets copies
+// and MMAs in flight land, writes expert -1 and gate 0 for its tokens, frees
+// its tensor memory and exits.
 #include "common.cuh"
 #include "internal.h"
 #include "tmap.h"
@@ -43,23 +51,24 @@ namespace {
 
 constexpr int kRM = 128;                           // tokens per tile (MMA M)
 constexpr int kRK = kTmapBoxK;                     // K elements per stage
-constexpr int kRThreads = 192;
-constexpr int kRMaxStages = 6;
+constexpr int kRMaxStages = 8;
 constexpr uint32_t kXTileBytes = kRM * kRK * 2;    // 16 KB of bf16 tokens per stage
 constexpr int kRouteTcMaxE = 160;                  // 3 * E_pad <= 512 TMEM columns
+constexpr int kRouteTcMaxK = 32;                   // pick scratch: k floats per token
 constexpr size_t kRouteSmemBudget = 110 * 1024;    // per CTA: two CTAs fit on an SM
+constexpr size_t kRpSmemBudget = 225 * 1024;       // per CTA when one fills the SM
 
 // Status word for callers that pass none (moe_route): waits still need one.
 __device__ uint32_t g_route_status_scratch;
 
 struct RouteTcArgs {
-    const float *W_g;
     const float *b_g;
     const float *noise;
     float sigma;
     int64_t N;
     int d, E, k, stages;
-    int splits;  // CTAs per token tile (a cluster), each summing one piece of K
+    int splits;    // S: pieces of K
+    int pick_off;  // byte offset of the pick scratch: k floats per token row of a tile
     float *logits_out;
     int32_t *topk_idx;
     float *gates;
@@ -115,28 +124,219 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int UPT>  // E_pad = 16 * UPT experts per part
-__host__ __device__ constexpr uint32_t route_tmem_cols() {
-    return 3 * 16 * UPT <= 64 ? 64 : 3 * 16 * UPT <= 128 ? 128 : 3 * 16 * UPT <= 256 ? 256 : 512;
+template <int UPT>
+__host__ __device__ constexpr int route_nb() {  // rows of B = accumulator columns
+    return 3 * 16 * UPT;
+}
+
+// One ring stage: the x tile (bf16, 128-byte swizzle), the B slot (3 * E_pad
+// bf16 rows, 128-byte swizzle) and, for the in-kernel split, the fp32 W_g tile
+// the B slot is split from (E_pad rows of 64, unswizzled, zero past E).
+template <int UPT>
+__host__ __device__ constexpr uint32_t route_b_bytes() {
+    return static_cast<uint32_t>(route_nb<UPT>()) * kRK * 2u;
+}
+template <int UPT, bool PRE>
+__host__ __device__ constexpr uint32_t route_wtile_bytes() {
+    return PRE ? 0u : 16u * UPT * kRK * 4u;
+}
+template <int UPT, bool PRE>
+__host__ __device__ constexpr uint32_t route_stage_bytes() {
+    return kXTileBytes + route_b_bytes<UPT>() + route_wtile_bytes<UPT, PRE>();
+}
+// Rows of B per TMA box when pre-split (a box holds at most 256 rows).
+template <int UPT>
+__host__ __device__ constexpr int route_b_box_rows() {
+    return route_nb<UPT>() <= 256 ? route_nb<UPT>() : route_nb<UPT>() / 2;
+}
+
+// TMA loads of one stage: the x tile of rows row0.. and K block kb, and B
+// (pre-split) or the fp32 W_g tile (in-kernel split), all on barrier `bar`.
+template <int UPT, bool PRE>
+__device__ __forceinline__ void load_stage(uint32_t st, const CUtensorMap *tm_x, const CUtensorMap *tm_w,
+                                           uint32_t bar, int kb, int row0) {
+    mbar_arrive_expect_tx(bar, kXTileBytes + (PRE ? route_b_bytes<UPT>() : route_wtile_bytes<UPT, PRE>()));
+    tma_load_2d(st, tm_x, bar, kb * kRK, row0);
+    if constexpr (PRE) {
+        constexpr int box = route_b_box_rows<UPT>();
+#pragma unroll
+        for (int r = 0; r < route_nb<UPT>(); r += box)
+            tma_load_2d(st + kXTileBytes + static_cast<uint32_t>(r) * 128u, tm_w, bar, kb * kRK, r);
+    } else {
+        tma_load_2d(st + kXTileBytes + route_b_bytes<UPT>(), tm_w, bar, kb * kRK, 0);
+    }
+}
+
+// In-kernel split of the fp32 W_g tile of one stage into its B slot.  Thread
+// et (0..127) of the splitting warps owns units et + 128 i: expert row u / 8,
+// 8-column chunk u % 8.
+template <int UPT>
+__device__ __forceinline__ void split_stage(uint8_t *stage_gen, int et) {
+    constexpr int E_PAD = 16 * UPT;
+    const float *wt = reinterpret_cast<const float *>(stage_gen + kXTileBytes + route_b_bytes<UPT>());
+    uint8_t *bbase = stage_gen + kXTileBytes;
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+        const int u = et + i * 128;
+        const int e = u >> 3, c = u & 7;
+        const float4 a = *reinterpret_cast<const float4 *>(wt + e * kRK + c * 8);
+        const float4 b = *reinterpret_cast<const float4 *>(wt + e * kRK + c * 8 + 4);
+        uint4 hi, mid, lo;
+        split3(a.x, a.y, hi.x, mid.x, lo.x);
+        split3(a.z, a.w, hi.y, mid.y, lo.y);
+        split3(b.x, b.y, hi.z, mid.z, lo.z);
+        split3(b.z, b.w, hi.w, mid.w, lo.w);
+        *reinterpret_cast<uint4 *>(bbase + sw128_offset(e, c)) = hi;
+        *reinterpret_cast<uint4 *>(bbase + sw128_offset(E_PAD + e, c)) = mid;
+        *reinterpret_cast<uint4 *>(bbase + sw128_offset(2 * E_PAD + e, c)) = lo;
+    }
+}
+
+// Pre-split of all of W_g: w3[p * E_pad + e][c] = part p of W_g[e][c], zero for
+// e >= E.  One thread per 8 columns of one expert row.
+__global__ void __launch_bounds__(256)
+route_split_kernel(const float *__restrict__ W_g, int E, int E_pad, int d, __nv_bfloat16 *__restrict__ w3) {
+    pdl_trigger();
+    pdl_wait();
+    const int chunks = d / 8;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<int64_t>(E_pad) * chunks) return;
+    const int e = static_cast<int>(i / chunks), c = static_cast<int>(i % chunks) * 8;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (e < E) {
+        const float4 *p = reinterpret_cast<const float4 *>(W_g + static_cast<int64_t>(e) * d + c);
+        a = p[0];
+        b = p[1];
+    }
+    uint4 hi, mid, lo;
+    split3(a.x, a.y, hi.x, mid.x, lo.x);
+    split3(a.z, a.w, hi.y, mid.y, lo.y);
+    split3(b.x, b.y, hi.z, mid.z, lo.z);
+    split3(b.z, b.w, hi.w, mid.w, lo.w);
+    const int64_t plane = static_cast<int64_t>(E_pad) * d;
+    uint4 *o = reinterpret_cast<uint4 *>(w3 + static_cast<int64_t>(e) * d + c);
+    o[0] = hi;
+    *reinterpret_cast<uint4 *>(w3 + plane + static_cast<int64_t>(e) * d + c) = mid;
+    *reinterpret_cast<uint4 *>(w3 + 2 * plane + static_cast<int64_t>(e) * d + c) = lo;
 }
 
 template <int UPT>
-__host__ __device__ constexpr uint32_t route_stage_bytes() {
-    return kXTileBytes + 3u * 16u * UPT * kRK * 2u;
+__host__ __device__ constexpr uint32_t route_tmem_cols() {  // clustered: one buffer
+    return route_nb<UPT>() <= 64 ? 64 : route_nb<UPT>() <= 128 ? 128 : route_nb<UPT>() <= 256 ? 256 : 512;
+}
+template <int UPT>
+__host__ __device__ constexpr uint32_t routep_tmem_cols() {  // persistent: two buffers
+    return 2 * route_nb<UPT>() <= 128 ? 128 : 2 * route_nb<UPT>() <= 256 ? 256 : 512;
 }
 
-// Which K blocks CTA `c` of an S-CTA cluster sums: [c*kb/S, (c+1)*kb/S).
+// Which K blocks piece c of S sums: [c*kb/S, (c+1)*kb/S).
 __host__ __device__ inline int route_kb_begin(int c, int S, int kb_total) {
     return static_cast<int>(static_cast<int64_t>(c) * kb_total / S);
 }
 
-// CTAs per token tile: the K range is cut into S pieces of at least 8 blocks
-// (512 columns), S <= 8.  S depends on d only, so a token's logits do not
-// depend on the batch size or on where the token sits in the batch.
+// Pieces of K: at least 8 blocks (512 columns) each, at most 8.  S depends
+// on d only.
 __host__ __device__ inline int route_k_splits(int d) {
     const int kb_total = (d + kRK - 1) / kRK;
     const int s = (kb_total + 7) / 8;
     return s < 1 ? 1 : (s > 8 ? 8 : s);
+}
+
+// MMAs of one stage into accumulator d_tmem (N = 3 * E_pad, issued in chunks
+// of at most 256 columns); acc0 = 0 starts the sum.
+template <int UPT>
+__device__ __forceinline__ void mma_stage(uint32_t st, uint32_t d_tmem, bool acc0) {
+    constexpr int NB = route_nb<UPT>();
+    const uint64_t ad = smem_desc_sw128(st);
+#pragma unroll
+    for (int kk = 0; kk < kRK / 16; ++kk) {
+#pragma unroll
+        for (int n0 = 0; n0 < NB; n0 += 256) {
+            constexpr int kChunk = NB < 256 ? NB : 256;
+            const int nn = (NB - n0) < kChunk ? (NB - n0) : kChunk;
+            const uint64_t bd = smem_desc_sw128(st + kXTileBytes + static_cast<uint32_t>(n0) * 128u);
+            // +32 bytes along K inside the swizzled row = +2 in the address field
+            umma_bf16(d_tmem + static_cast<uint32_t>(n0), ad + 2 * kk, bd + 2 * kk, idesc_bf16_f32(kRM, nn),
+                      (!acc0 || kk > 0) ? 1u : 0u);
+        }
+    }
+}
+
+// Sum of one piece for this thread's token row: (hi + mid) + lo per expert,
+// from accumulator columns taddr (+E_pad, +2 E_pad); run = piece sum (first
+// piece) or run + piece sum.
+template <int UPT>
+__device__ __forceinline__ void drain_piece(uint32_t taddr, bool first, float (&run)[16 * UPT]) {
+    constexpr int E_PAD = 16 * UPT;
+#pragma unroll
+    for (int ch = 0; ch < UPT; ++ch) {
+        uint32_t h[16], m[16], l[16];
+        tmem_ld_32x32b_x16(taddr + ch * 16, h);
+        tmem_ld_32x32b_x16(taddr + E_PAD + ch * 16, m);
+        tmem_ld_32x32b_x16(taddr + 2 * E_PAD + ch * 16, l);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float p = __fadd_rn(__fadd_rn(__uint_as_float(h[i]), __uint_as_float(m[i])), __uint_as_float(l[i]));
+            run[ch * 16 + i] = first ? p : __fadd_rn(run[ch * 16 + i], p);
+        }
+    }
+}
+
+// KeepTopK and softmax of one token (one thread): k rounds, each taking the
+// best score ranked after the previous pick (score descending, lower expert
+// index first on ties); then the softmax over the kept scores.  pv_s: this
+// thread's k floats of scratch.  Scores in shared memory (sr[0..E)).
+__device__ __forceinline__ void pick_row_smem(const float *sr, int E, int k, float *pv_s, int32_t *ti, float *gt) {
+    float pv = 0.0f;
+    int pe = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = 0.0f;
+        int be = -1;
+        for (int e = 0; e < E; ++e) {
+            const float v = sr[e];
+            if ((pe < 0 || ranks_before_tc(pv, pe, v, e)) && (be < 0 || ranks_before_tc(v, e, bv, be))) {
+                bv = v;
+                be = e;
+            }
+        }
+        ti[j] = be;
+        pv_s[j] = bv;
+        pv = bv;
+        pe = be;
+    }
+    const float mx = pv_s[0];
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(pv_s[j], mx)));
+    for (int j = 0; j < k; ++j) gt[j] = __fdiv_rn(expf(__fsub_rn(pv_s[j], mx)), sum);
+}
+
+// The same for scores held in registers (s[0..E), E <= E_PAD).
+template <int E_PAD>
+__device__ __forceinline__ void pick_row_regs(const float (&s)[E_PAD], int E, int k, float *pv_s, int32_t *ti,
+                                              float *gt) {
+    float pv = 0.0f;
+    int pe = -1;
+    for (int j = 0; j < k; ++j) {
+        float bv = 0.0f;
+        int be = -1;
+#pragma unroll
+        for (int e = 0; e < E_PAD; ++e) {
+            if (e < E && (pe < 0 || ranks_before_tc(pv, pe, s[e], e)) &&
+                (be < 0 || ranks_before_tc(s[e], e, bv, be))) {
+                bv = s[e];
+                be = e;
+            }
+        }
+        ti[j] = be;
+        pv_s[j] = bv;
+        pv = bv;
+        pe = be;
+    }
+    const float mx = pv_s[0];
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(pv_s[j], mx)));
+    for (int j = 0; j < k; ++j) gt[j] = __fdiv_rn(expf(__fsub_rn(pv_s[j], mx)), sum);
 }
 
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
@@ -150,15 +350,23 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
     return v;
 }
 
-template <int UPT>
-__global__ void __launch_bounds__(kRThreads, 1)
-route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args) {
+// ------------------------------------------------------------------ clustered form
+// Cluster of S CTAs per token tile; CTA c sums piece c of K.  Warp roles (192
+// threads): warp 0 lane 0 issues the TMA loads into a STAGES-deep ring; warp 1
+// owns the tensor memory and its lane 0 issues the MMAs; warps 2-5 split W_g
+// into the B slots (in-kernel split only), then write this piece's sums to a
+// table in shared memory.  After a cluster barrier CTA c finishes rows
+// [c*128/S, (c+1)*128/S) of the tile: adds the S tables in piece order
+// (reading the others through distributed shared memory), the bias, writes
+// the logits, adds the noise, picks and normalises.
+template <int UPT, bool PRE>
+__global__ void __launch_bounds__(192, (PRE || UPT <= 2) ? 2 : 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                const RouteTcArgs args) {
     constexpr int E_PAD = 16 * UPT;
-    constexpr int NB = 3 * E_PAD;                    // rows of B
-    constexpr uint32_t STAGE = route_stage_bytes<UPT>();
+    constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
     constexpr uint32_t TMEM_COLS = route_tmem_cols<UPT>();
     static_assert(STAGE % 1024 == 0, "stage alignment");
-    static_assert(NB <= 512, "accumulator columns");
 
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 2];
@@ -169,7 +377,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
     const int stages = args.stages;
     const int E = args.E, d = args.d, k = args.k;
     const int kb_total = (d + kRK - 1) / kRK;
-    const int S = args.splits;                      // CTAs of this cluster, one K piece each
+    const int S = args.splits;
     const int crank = static_cast<int>(cluster_ctarank());
     const int kb0 = route_kb_begin(crank, S, kb_total), kb1 = route_kb_begin(crank + 1, S, kb_total);
     const int64_t t0 = static_cast<int64_t>(blockIdx.x / S) * kRM;
@@ -178,8 +386,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
 
     const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
-    const uint32_t xfull0 = smem_u32(&bars[0]);                 // x tile landed (TMA bytes)
-    const uint32_t wfull0 = smem_u32(&bars[kRMaxStages]);       // W parts written (4 warps)
+    const uint32_t xfull0 = smem_u32(&bars[0]);                 // stage loaded (TMA bytes)
+    const uint32_t wfull0 = smem_u32(&bars[kRMaxStages]);       // B slot split (4 warps)
     const uint32_t empty0 = smem_u32(&bars[2 * kRMaxStages]);   // MMAs done with the stage
     const uint32_t accf = smem_u32(&bars[3 * kRMaxStages]);     // accumulator final
     const uint32_t drain = smem_u32(&bars[3 * kRMaxStages + 1]);
@@ -195,7 +403,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
         fence_barrier_init();
         epi_fail = 0;
     }
-    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_x);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w);
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
         tmem_relinquish();
@@ -211,7 +422,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer (x tiles)
+        // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int stage = 0, issued = 0;
             uint32_t phase = 0;
@@ -221,9 +432,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
                     ok = false;
                     break;
                 }
-                const uint32_t fb = xfull0 + 8 * stage;
-                mbar_arrive_expect_tx(fb, kXTileBytes);
-                tma_load_2d(smem_base + stage * STAGE, &tm_x, fb, kb * kRK, static_cast<int>(t0));
+                load_stage<UPT, PRE>(smem_base + stage * STAGE, &tm_x, &tm_w, xfull0 + 8 * stage, kb,
+                                     static_cast<int>(t0));
                 ++issued;
                 if (++stage == stages) {
                     stage = 0;
@@ -251,27 +461,14 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, any = false;
-            for (int kb = kb0; kb < kb1 && ok; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb) {
                 if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 12) ||
-                    !mbar_wait_bounded(wfull0 + 8 * stage, phase, status, tmo, 13)) {
+                    (!PRE && !mbar_wait_bounded(wfull0 + 8 * stage, phase, status, tmo, 13))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sa = smem_base + stage * STAGE;
-                const uint64_t ad = smem_desc_sw128(sa);
-#pragma unroll
-                for (int kk = 0; kk < kRK / 16; ++kk) {
-#pragma unroll
-                    for (int n0 = 0; n0 < NB; n0 += 256) {
-                        constexpr int kChunk = NB < 256 ? NB : 256;
-                        const int nn = (NB - n0) < kChunk ? (NB - n0) : kChunk;
-                        const uint64_t bd = smem_desc_sw128(sa + kXTileBytes + static_cast<uint32_t>(n0) * 128u);
-                        // +32 bytes along K inside the swizzled row = +2 in the address field
-                        umma_bf16(tmem_base + static_cast<uint32_t>(n0), ad + 2 * kk, bd + 2 * kk,
-                                  idesc_bf16_f32(kRM, nn), (kb > kb0 || kk > 0) ? 1u : 0u);
-                    }
-                }
+                mma_stage<UPT>(smem_base + stage * STAGE, tmem_base, kb == kb0);
                 any = true;
                 umma_commit(empty0 + 8 * stage);
                 if (++stage == stages) {
@@ -287,50 +484,20 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
             }
         }
     } else {
-        // ------------------------------------------------ W_g split, then this K piece's sums
+        // ------------------------------------------------ W_g split, then this piece's sums
         const int et = threadIdx.x - 64;  // 0..127
         const int q = warp & 3;           // TMEM lane quarter this warp may read
         const int row = q * 32 + lane;
         bool ok = true;
-        {
+        if constexpr (!PRE) {
             int stage = 0;
             uint32_t phase = 0;
             for (int kb = kb0; kb < kb1; ++kb) {
-                // this K block's weights, loaded before the slot frees up
-                float w[UPT][8];
-                const int col0 = kb * kRK;
-#pragma unroll
-                for (int i = 0; i < UPT; ++i) {
-                    const int u = et + i * 128;
-                    const int e = u >> 3, col = col0 + (u & 7) * 8;
-                    if (e < E && col < d) {
-                        const float4 *p = reinterpret_cast<const float4 *>(args.W_g + static_cast<int64_t>(e) * d + col);
-                        const float4 a = p[0], b = p[1];
-                        w[i][0] = a.x; w[i][1] = a.y; w[i][2] = a.z; w[i][3] = a.w;
-                        w[i][4] = b.x; w[i][5] = b.y; w[i][6] = b.z; w[i][7] = b.w;
-                    } else {
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) w[i][v] = 0.0f;
-                    }
-                }
-                if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 14)) {
+                if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 14)) {
                     ok = false;
                     break;
                 }
-                uint8_t *bbase = smem_gen + stage * STAGE + kXTileBytes;
-#pragma unroll
-                for (int i = 0; i < UPT; ++i) {
-                    const int u = et + i * 128;
-                    const int e = u >> 3, c = u & 7;
-                    uint4 hi, mid, lo;
-                    split3(w[i][0], w[i][1], hi.x, mid.x, lo.x);
-                    split3(w[i][2], w[i][3], hi.y, mid.y, lo.y);
-                    split3(w[i][4], w[i][5], hi.z, mid.z, lo.z);
-                    split3(w[i][6], w[i][7], hi.w, mid.w, lo.w);
-                    *reinterpret_cast<uint4 *>(bbase + sw128_offset(e, c)) = hi;
-                    *reinterpret_cast<uint4 *>(bbase + sw128_offset(E_PAD + e, c)) = mid;
-                    *reinterpret_cast<uint4 *>(bbase + sw128_offset(2 * E_PAD + e, c)) = lo;
-                }
+                split_stage<UPT>(smem_gen + stage * STAGE, et);
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wfull0 + 8 * stage);
@@ -345,8 +512,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (ok) {
-            // this piece's sum per (token, expert): (hi + mid) + lo, into the
-            // partial table [128][ld] that reuses the ring
+            // this piece's sum per (token, expert) into the table [128][ld]
+            // that reuses the ring
             const int ld = E + 1 + (E & 1);  // odd row stride: conflict-free column access
             float *part = reinterpret_cast<float *>(smem_gen);
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -370,14 +537,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
         }
     }
     tc_fence_before();
-    cluster_sync();  // every piece's partial table and failure flag is in place
+    cluster_sync();  // every piece's table and failure flag is in place
 
     if (warp >= 2) {
         // ------------------------------------------------ this CTA's token rows
-        // CTA c of the cluster finishes rows [c*128/S, (c+1)*128/S) of the tile:
-        // adds the S partial sums in piece order, the bias, writes the logits,
-        // adds the noise, then picks and normalises.  Its own rows of its own
-        // table are read by nobody else, so the final scores go there.
+        // Its own rows of its own table are read by nobody else, so the final
+        // scores go there.
         const int et = threadIdx.x - 64;
         const int ld = E + 1 + (E & 1);
         float *part = reinterpret_cast<float *>(smem_gen);
@@ -394,6 +559,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
         if (good) {
             const int64_t base = (t0 + r0) * E;
             const int total = nrows * E;
+#pragma unroll 4
             for (int i = et; i < total; i += 128) {
                 const int r = r0 + i / E, e = i % E;
                 const uint32_t off = static_cast<uint32_t>(r * ld + e) * 4u;
@@ -412,29 +578,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
             int32_t *ti = args.topk_idx + t * k;
             float *gt = args.gates + t * k;
             if (good) {
-                // k rounds: the best score ranked after the previous pick
-                const float *sr = part + r * ld;
-                float pv = 0.0f;
-                int pe = -1;
-                for (int j = 0; j < k; ++j) {
-                    float bv = 0.0f;
-                    int be = -1;
-                    for (int e = 0; e < E; ++e) {
-                        const float v = sr[e];
-                        if ((pe < 0 || ranks_before_tc(pv, pe, v, e)) && (be < 0 || ranks_before_tc(v, e, bv, be))) {
-                            bv = v;
-                            be = e;
-                        }
-                    }
-                    ti[j] = be;
-                    gt[j] = bv;  // the kept score, until the softmax below replaces it
-                    pv = bv;
-                    pe = be;
-                }
-                const float mx = gt[0];
-                float sum = 0.0f;
-                for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(gt[j], mx)));
-                for (int j = 0; j < k; ++j) gt[j] = __fdiv_rn(expf(__fsub_rn(gt[j], mx)), sum);
+                pick_row_smem(part + r * ld, E, k, reinterpret_cast<float *>(smem_gen + args.pick_off) + et * k, ti, gt);
             } else {
                 for (int j = 0; j < k; ++j) {
                     ti[j] = -1;
@@ -450,19 +594,272 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const RouteTcArgs args
     }
 }
 
-template <int UPT>
-cudaError_t launch_route_tc_t(const CUtensorMap &tm, RouteTcArgs a, int64_t tiles, cudaStream_t s) {
-    constexpr uint32_t STAGE = route_stage_bytes<UPT>();
-    int stages = static_cast<int>((kRouteSmemBudget - 1024) / STAGE);
-    if (stages > kRMaxStages) stages = kRMaxStages;
-    if (stages < 2) stages = 2;
-    const size_t ring = static_cast<size_t>(stages) * STAGE;
-    const int ld = a.E + 1 + (a.E & 1);
-    if (static_cast<size_t>(kRM) * ld * sizeof(float) > ring) return cudaErrorInvalidValue;
-    const size_t smem = ring + 1024;
-    a.stages = stages;
-    a.splits = route_k_splits(a.d);
-    auto kern = route_tc_kernel<UPT>;
+// ------------------------------------------------------------------ persistent form
+// One CTA per SM walks tiles tile = blockIdx.x, + gridDim.x, ...; the ring and
+// the MMAs run on from one tile to the next.  Each piece of a tile sums from
+// zero into one of two tensor-memory buffers; the epilogue adds the piece sums
+// in order in registers, so each token gets what the clustered form gives it.
+//
+// Warp roles: warp 0 lane 0 loads stages by TMA; warp 1 owns the tensor
+// memory and its lane 0 issues the MMAs; warps 2-5 drain the accumulators
+// (one token row per thread) and finish each tile (bias, logits, noise,
+// KeepTopK, softmax); warps 6-9 (in-kernel split only) split W_g into the B
+// slots.
+template <bool PRE>
+__host__ __device__ constexpr int routep_threads() {
+    return PRE ? 192 : 320;
+}
+
+template <int UPT, bool PRE>
+__global__ void __launch_bounds__(routep_threads<PRE>(), 1)
+route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                 const RouteTcArgs args) {
+    constexpr int E_PAD = 16 * UPT;
+    constexpr int NB = route_nb<UPT>();
+    constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
+    constexpr uint32_t TMEM_COLS = routep_tmem_cols<UPT>();
+    static_assert(2 * NB <= 512, "two accumulator buffers");
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 5];
+    __shared__ uint32_t tmem_holder;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int stages = args.stages;
+    const int E = args.E, d = args.d, k = args.k;
+    const int kb_total = (d + kRK - 1) / kRK;
+    const int S = args.splits;
+    const int64_t tiles = (args.N + kRM - 1) / kRM;
+    const uint64_t tmo = args.timeout_ns;
+    uint32_t *status = args.status != nullptr ? args.status : &g_route_status_scratch;
+
+    const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
+    const uint32_t xfull0 = smem_u32(&bars[0]);
+    const uint32_t wfull0 = smem_u32(&bars[kRMaxStages]);
+    const uint32_t empty0 = smem_u32(&bars[2 * kRMaxStages]);
+    const uint32_t accf0 = smem_u32(&bars[3 * kRMaxStages]);      // [2] piece sum ready
+    const uint32_t acce0 = smem_u32(&bars[3 * kRMaxStages + 2]);  // [2] buffer drained
+    const uint32_t drain = smem_u32(&bars[3 * kRMaxStages + 4]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(xfull0 + 8 * s, 1);
+            mbar_init(wfull0 + 8 * s, 4);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf0 + 8 * b, 1);
+            mbar_init(acce0 + 8 * b, 4);
+        }
+        mbar_init(drain, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_trigger();  // after the tensor memory is held (see the clustered form)
+    const uint32_t tmem_base = tmem_holder;
+    pdl_wait();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 21)) {
+                        ok = false;
+                        break;
+                    }
+                    load_stage<UPT, PRE>(smem_base + stage * STAGE, &tm_x, &tm_w, xfull0 + 8 * stage, kb,
+                                         static_cast<int>(tile * kRM));
+                    ++issued;
+                    if (++stage == stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < stages && i < issued; ++i) {
+                    if (st == 0) {
+                        st = stages - 1;
+                        ph ^= 1u;
+                    } else {
+                        --st;
+                    }
+                    wait_until(xfull0 + 8 * st, ph, tmo);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int piece = 0;  // pieces issued by this CTA so far
+            bool ok = true, any = false;
+            for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                for (int c = 0; c < S && ok; ++c, ++piece) {
+                    const int b = piece & 1;
+                    const uint32_t use = static_cast<uint32_t>(piece >> 1);
+                    if (!mbar_wait_bounded(acce0 + 8 * b, (use & 1u) ^ 1u, status, tmo, 22)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kb0 = route_kb_begin(c, S, kb_total), kb1 = route_kb_begin(c + 1, S, kb_total);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * NB);
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 23) ||
+                            (!PRE && !mbar_wait_bounded(wfull0 + 8 * stage, phase, status, tmo, 24))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        mma_stage<UPT>(smem_base + stage * STAGE, d_tmem, kb == kb0);
+                        any = true;
+                        umma_commit(empty0 + 8 * stage);
+                        if (++stage == stages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (ok) umma_commit(accf0 + 8 * b);
+                }
+            }
+            if (!ok && any) {
+                umma_commit(drain);
+                wait_until(drain, 0, tmo);
+            }
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------ W_g split into the B slots
+        if constexpr (!PRE) {
+            const int et = threadIdx.x - 192;  // 0..127
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < kb_total; ++kb) {
+                    if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 25)) {
+                        ok = false;
+                        break;
+                    }
+                    split_stage<UPT>(smem_gen + stage * STAGE, et);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(wfull0 + 8 * stage);
+                    if (++stage == stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2-5)
+        const int q = warp & 3;    // TMEM lane quarter
+        const int row = q * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        float *pick_s = reinterpret_cast<float *>(smem_gen + args.pick_off);  // [128][k]
+        const bool use_noise = (args.noise != nullptr) && (args.sigma != 0.0f);
+        int piece = 0;
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            float run[E_PAD];
+            for (int c = 0; c < S; ++c, ++piece) {
+                const int b = piece & 1;
+                const uint32_t use = static_cast<uint32_t>(piece >> 1);
+                if (ok) ok = mbar_wait_bounded(accf0 + 8 * b, use & 1u, status, tmo, 26);
+                ok = __all_sync(0xffffffffu, ok);
+                tc_fence_after();
+                if (ok) drain_piece<UPT>(tmem_base + lane_off + static_cast<uint32_t>(b * NB), c == 0, run);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce0 + 8 * b);
+            }
+            // finish this thread's token: bias, logits out, noise, KeepTopK, softmax
+            const int64_t t = tile * kRM + row;
+            if (t < args.N) {
+                int32_t *ti = args.topk_idx + t * k;
+                float *gt = args.gates + t * k;
+                if (ok) {
+                    if (args.b_g) {
+#pragma unroll
+                        for (int e = 0; e < E_PAD; ++e)
+                            if (e < E) run[e] = __fadd_rn(run[e], args.b_g[e]);
+                    }
+                    const bool vec4 = (E & 3) == 0;  // rows of E floats are 16-byte aligned
+                    if (args.logits_out) {
+                        float *lo = args.logits_out + t * E;
+#pragma unroll
+                        for (int e = 0; e < E_PAD; e += 4) {
+                            if (vec4) {
+                                if (e < E)
+                                    *reinterpret_cast<float4 *>(lo + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+                            } else {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v)
+                                    if (e + v < E) lo[e + v] = run[e + v];
+                            }
+                        }
+                    }
+                    if (use_noise) {
+                        const float *nz = args.noise + t * E;
+#pragma unroll
+                        for (int e = 0; e < E_PAD; e += 4) {
+                            float q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                            if (vec4) {
+                                if (e < E) {
+                                    const float4 f = *reinterpret_cast<const float4 *>(nz + e);
+                                    q[0] = f.x; q[1] = f.y; q[2] = f.z; q[3] = f.w;
+                                }
+                            } else {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v)
+                                    if (e + v < E) q[v] = nz[e + v];
+                            }
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                if (e + v < E) run[e + v] = __fadd_rn(run[e + v], __fmul_rn(args.sigma, q[v]));
+                        }
+                    }
+                    pick_row_regs<E_PAD>(run, E, k, pick_s + row * k, ti, gt);
+                } else {
+                    for (int j = 0; j < k; ++j) {
+                        ti[j] = -1;
+                        gt[j] = 0.0f;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+template <int UPT, bool PRE, int KIND>  // KIND: 0 clustered, 1 persistent
+cudaError_t set_smem_attr(void (*kern)(CUtensorMap, CUtensorMap, RouteTcArgs), size_t smem) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -473,9 +870,32 @@ cudaError_t launch_route_tc_t(const CUtensorMap &tm, RouteTcArgs a, int64_t tile
         if (e != cudaSuccess) return e;
         attr_done.fetch_or(bit);
     }
+    return cudaSuccess;
+}
+
+template <int UPT, bool PRE>
+cudaError_t launch_cluster_t(const CUtensorMap &tm, const CUtensorMap &tw, RouteTcArgs a, int64_t tiles,
+                             cudaStream_t s) {
+    constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
+    // two CTAs per SM when two stages fit the half budget, else one CTA with
+    // as many stages as fit (one at least)
+    const size_t budget = (2 * STAGE + 1024 <= kRouteSmemBudget) ? kRouteSmemBudget : kRpSmemBudget;
+    int stages = static_cast<int>((budget - 1024) / STAGE);
+    if (stages > kRMaxStages) stages = kRMaxStages;
+    if (stages < 1) return cudaErrorInvalidValue;
+    const size_t ring = static_cast<size_t>(stages) * STAGE;
+    const int ld = a.E + 1 + (a.E & 1);
+    const size_t part_bytes = align_up(static_cast<size_t>(kRM) * ld * sizeof(float), 16);
+    if (part_bytes + static_cast<size_t>(kRM) * a.k * sizeof(float) > ring) return cudaErrorInvalidValue;
+    const size_t smem = ring + 1024;
+    a.stages = stages;
+    a.pick_off = static_cast<int>(part_bytes);
+    auto kern = route_tc_kernel<UPT, PRE>;
+    cudaError_t e = set_smem_attr<UPT, PRE, 0>(kern, smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * a.splits));
-    cfg.blockDim = dim3(kRThreads);
+    cfg.blockDim = dim3(192);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -487,34 +907,115 @@ cudaError_t launch_route_tc_t(const CUtensorMap &tm, RouteTcArgs a, int64_t tile
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, tm, a);
+    return cudaLaunchKernelEx(&cfg, kern, tm, tw, a);
+}
+
+template <int UPT, bool PRE>
+cudaError_t launch_persistent_t(const CUtensorMap &tm, const CUtensorMap &tw, RouteTcArgs a, int64_t tiles,
+                                int sms, cudaStream_t s) {
+    constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
+    const size_t pick_bytes = static_cast<size_t>(kRM) * a.k * sizeof(float);
+    const size_t fixed = pick_bytes + 1024;
+    if (fixed + STAGE > kRpSmemBudget) return cudaErrorInvalidValue;
+    int stages = static_cast<int>((kRpSmemBudget - fixed) / STAGE);
+    if (stages > kRMaxStages) stages = kRMaxStages;
+    const size_t ring = static_cast<size_t>(stages) * STAGE;
+    const size_t smem = ring + fixed;
+    a.stages = stages;
+    a.pick_off = static_cast<int>(ring);
+    auto kern = route_tcp_kernel<UPT, PRE>;
+    cudaError_t e = set_smem_attr<UPT, PRE, 1>(kern, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = tiles < sms ? tiles : sms;
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(routep_threads<PRE>()), smem, s, tm, tw, a);
+}
+
+template <int UPT, bool PRE>
+cudaError_t launch_form(bool persistent, const CUtensorMap &tm, const CUtensorMap &tw, const RouteTcArgs &a,
+                        int64_t tiles, int sms, cudaStream_t s) {
+    if constexpr (2 * route_nb<UPT>() <= 512) {
+        if (persistent) return launch_persistent_t<UPT, PRE>(tm, tw, a, tiles, sms, s);
+    }
+    return launch_cluster_t<UPT, PRE>(tm, tw, a, tiles, s);
+}
+
+template <bool PRE>
+cudaError_t launch_upt(int upt, bool persistent, const CUtensorMap &tm, const CUtensorMap &tw, const RouteTcArgs &a,
+                       int64_t tiles, int sms, cudaStream_t s) {
+    switch (upt) {
+        case 1: return launch_form<1, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 2: return launch_form<2, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 4: return launch_form<4, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 5: return launch_form<5, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 6: return launch_form<6, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 8: return launch_form<8, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        case 10: return launch_form<10, PRE>(persistent, tm, tw, a, tiles, sms, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// E_pad / 16 for E experts: the same value everywhere a given E is routed.
+int route_upt(int E) {
+    return E <= 16 ? 1 : E <= 32 ? 2 : E <= 64 ? 4 : E <= 80 ? 5 : E <= 96 ? 6 : E <= 128 ? 8 : 10;
+}
+
+// MOE_ROUTE_TCP=0 keeps large batches on the clustered form (for comparisons).
+bool route_tcp_enabled() {
+    static const bool enabled = [] {
+        const char *v = getenv("MOE_ROUTE_TCP");
+        return v == nullptr || atoi(v) != 0;
+    }();
+    return enabled;
 }
 
 }  // namespace
 
-bool route_tc_eligible(const void *x, const float *W_g, int64_t N, int d, int E) {
+bool route_tc_shape_ok(int64_t N, int d, int E, int k) {
     static const bool enabled = [] {
         const char *v = getenv("MOE_ROUTE_TC");
         return v == nullptr || atoi(v) != 0;
     }();
     return enabled && N > 0 && N < (static_cast<int64_t>(1) << 31) / 8 && d % 8 == 0 && E >= 1 &&
-           E <= kRouteTcMaxE && reinterpret_cast<uintptr_t>(x) % 16 == 0 &&
+           E <= kRouteTcMaxE && k >= 1 && k <= kRouteTcMaxK;
+}
+
+bool route_tc_eligible(const void *x, const float *W_g, int64_t N, int d, int E, int k) {
+    return route_tc_shape_ok(N, d, E, k) && reinterpret_cast<uintptr_t>(x) % 16 == 0 &&
            reinterpret_cast<uintptr_t>(W_g) % 16 == 0;
+}
+
+size_t route_tc_w3_bytes(int d, int E) {
+    if (d < 1 || d % 8 != 0 || E < 1 || E > kRouteTcMaxE) return 0;
+    return align_up(static_cast<size_t>(3) * 16 * route_upt(E) * d * 2, 256);
 }
 
 cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, const float *noise, float sigma,
                             int64_t N, int d, int E, int k, float *logits_out, int32_t *topk_idx, float *gates,
-                            uint32_t *status, uint64_t timeout_ns, cudaStream_t s) {
-    CUtensorMap tm;
+                            uint32_t *status, uint64_t timeout_ns, void *w3, cudaStream_t s) {
+    CUtensorMap tm, tw;
     if (!make_tmap_bf16_2d(&tm, x, N, d, kRM)) return cudaErrorInvalidValue;
-    RouteTcArgs a{W_g, b_g, noise, sigma, N, d, E, k, 0, 1, logits_out, topk_idx, gates, status, timeout_ns};
+    const int upt = route_upt(E);
+    const int e_pad = 16 * upt, nb = 3 * e_pad;
+    if (w3 != nullptr) {
+        // the parts of all of W_g, then B by TMA
+        const int64_t units = static_cast<int64_t>(e_pad) * (d / 8);
+        cudaError_t e = launch_pdl(route_split_kernel, dim3(static_cast<unsigned>((units + 255) / 256)), dim3(256), 0,
+                                   s, W_g, E, e_pad, d, static_cast<__nv_bfloat16 *>(w3));
+        if (e != cudaSuccess) return e;
+        if (!make_tmap_bf16_2d(&tw, w3, nb, d, nb <= 256 ? nb : nb / 2)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_tmap_f32_2d(&tw, W_g, E, d, e_pad, kRK)) return cudaErrorInvalidValue;
+    }
+    RouteTcArgs a{b_g, noise, sigma, N, d, E, k, 0, route_k_splits(d), 0, logits_out, topk_idx, gates, status,
+                  timeout_ns};
     const int64_t tiles = (N + kRM - 1) / kRM;
-    if (E <= 16) return launch_route_tc_t<1>(tm, a, tiles, s);
-    if (E <= 32) return launch_route_tc_t<2>(tm, a, tiles, s);
-    if (E <= 64) return launch_route_tc_t<4>(tm, a, tiles, s);
-    if (E <= 96) return launch_route_tc_t<6>(tm, a, tiles, s);
-    if (E <= 128) return launch_route_tc_t<8>(tm, a, tiles, s);
-    return launch_route_tc_t<10>(tm, a, tiles, s);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // many tiles: the persistent form; few: clusters spread one tile's K over
+    // up to 8 SMs
+    const bool persistent = tiles * a.splits >= 2 * static_cast<int64_t>(sms) && route_tcp_enabled();
+    return w3 != nullptr ? launch_upt<true>(upt, persistent, tm, tw, a, tiles, sms, s)
+                         : launch_upt<false>(upt, persistent, tm, tw, a, tiles, sms, s);
 }
 
 }  // namespace moe

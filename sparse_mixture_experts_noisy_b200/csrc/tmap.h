@@ -16,4 +16,8 @@ bool make_tmap_bf16_2d(CUtensorMap *m, const void *base, int64_t rows, int K, in
 // [E, Nw, K] bf16, box = 64 (K) x box_rows x 1, 128-byte swizzle, zero fill.
 bool make_tmap_bf16_3d(CUtensorMap *m, const void *base, int E, int Nw, int K, int box_rows);
 
+// [rows, cols] row-major fp32, box = box_cols x box_rows, no swizzle, zero
+// fill past either edge (cols * 4 must be a multiple of 16).
+bool make_tmap_f32_2d(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows, int box_cols);
+
 }  // namespace moe

@@ -13,7 +13,7 @@ index) and softmax.
 The shapes cover one and two MMA column chunks (3 * E_pad up to 480 rows of
 B), odd expert counts, a K tail shorter than a 64-wide block, a last token
 tile of one row, exact ties between experts, and the CUDA-core fallback above
-160 experts."""
+160 experts or 32 choices."""
 import numpy as np
 import pytest
 import torch
@@ -40,6 +40,10 @@ SHAPES = {
     "e96_two_chunks": _wl("e96", N=1300, d=520, E=96, k=4, sigma=1.0, wg_std=0.05),
     "e160_largest": _wl("e160", N=1200, d=256, E=160, k=8, sigma=0.0, wg_std=1.0),
     "e161_fallback": _wl("e161", N=1050, d=64, E=161, k=2, sigma=0.0, wg_std=1.0),
+    "k33_fallback": _wl("k33", N=1100, d=64, E=40, k=33, sigma=0.5, wg_std=1.0),
+    # enough tiles for the persistent form
+    "e64_persistent": _wl("e64p", N=20000, d=2048, E=64, k=6, sigma=1.0),
+    "e80_persistent": _wl("e80p", N=40000, d=1024, E=80, k=4, sigma=0.5, wg_std=0.05, bias0=0.5),
 }
 
 
@@ -94,10 +98,18 @@ def test_router_ties_go_to_lower_index():
     assert ((idx == 6).any(1) <= (idx == 2).any(1)).all(), "expert 6 kept without its tied twin 2"
 
 
-def test_router_fused_forward_matches_staged():
-    """moe_forward routes through the same kernel as moe_route."""
+FWD_CASES = {
+    "clustered": Workload("fwd", BF16, N=2048, d=512, E=8, d_ff=256, k=2, sigma=1.0, cf=1.25, w_std=0.05),
+    "persistent": Workload("fwdp", BF16, N=20000, d=2048, E=64, d_ff=128, k=6, sigma=1.0, cf=1.0, w_std=0.05),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FWD_CASES))
+def test_router_fused_forward_matches_staged(name):
+    """moe_forward (router weights split once by a first pass, read by TMA)
+    and moe_route (split inside the router kernel) give the same bits."""
     require_gpu()
-    wl = Workload("fwd", BF16, N=2048, d=512, E=8, d_ff=256, k=2, sigma=1.0, cf=1.25, w_std=0.05)
+    wl = FWD_CASES[name]
     inp = make_inputs(wl, seed=23)
     x, W_g, noise = to_dev(inp.x), to_dev(inp.W_g), to_dev(inp.noise)
     topk, gates, logits = moe.moe_route(x, W_g, wl.k, noise=noise, sigma=wl.sigma)
@@ -115,6 +127,9 @@ BATCH_CASES = {
     "f32_cuda_cores": Workload("bi_f32", "f32", N=2100, d=1000, E=12, d_ff=16, k=3, sigma=0.5, cf=1.0,
                                wg_std=0.1),
     "bf16_cuda_cores": _wl("bi_odd", N=2100, d=36, E=5, k=2, sigma=0.0, wg_std=0.3),
+    # the whole batch takes the persistent form, the slices the clustered one
+    "bf16_persistent_e8": _wl("bi_p8", N=20000, d=4096, E=8, k=2, sigma=1.0, bias0=1.0),
+    "bf16_persistent_e64": _wl("bi_p64", N=20000, d=2048, E=64, k=6, sigma=1.0),
 }
 
 
@@ -130,7 +145,7 @@ def test_router_batch_size_independent(name):
     x, W_g, b_g, noise = to_dev(inp.x), to_dev(inp.W_g), to_dev(inp.b_g), to_dev(inp.noise)
     topk, gates, logits = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma)
     # even starts keep every slice 16-byte aligned (the ABI requires it)
-    for a, b in ((6, 7), (100, 164), (0, 1000), (8, 1033), (2, 2100)):
+    for a, b in ((6, 7), (100, 164), (0, 1000), (8, 1033), (2, min(2100, wl.N)), (2, wl.N - 1)):
         sl = slice(a, b)
         nz = None if noise is None else noise[sl].contiguous()
         t2, g2, l2 = moe.moe_route(x[sl].contiguous(), W_g, wl.k, b_g=b_g, noise=nz, sigma=wl.sigma)
