@@ -16,6 +16,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <cstdlib>
+
 namespace moe {
 
 namespace {
@@ -213,6 +215,83 @@ combine_token_kernel(const T *__restrict__ out_rows, const int32_t *__restrict__
     Vec<T, VEC>::store(y + t * d + c, acc);
 }
 
+// Large batches: one warp per token (grid-stride), the mirror of the gather.
+// Lanes j < k fetch the token's (row, gate) pairs once and pass them round by
+// shuffles.  Each pass loads U 16-byte chunks per lane of every kept row
+// before using any (k * U loads in flight per lane, kept packed), then forms
+// the weighted sums in choice order (the same arithmetic per element as the
+// kernels above) and stores U chunks of y.
+template <typename T, int VEC, int KMAX, int U>
+__global__ void __launch_bounds__(256, 3)
+combine_warp_kernel(const T *__restrict__ out_rows, const int32_t *__restrict__ slot,
+                    const int32_t *__restrict__ topk_idx, const int32_t *__restrict__ offsets,
+                    const float *__restrict__ gates, int64_t N, int d, int k, int E, T *__restrict__ y) {
+    using Raw = typename Vec<T, VEC>::Raw;
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int chunks = d / VEC;
+    for (int64_t t = w0; t < N; t += nw) {
+        int32_t row = -1;
+        float g = 0.0f;
+        if (lane < k) {
+            const int32_t sl = slot[t * k + lane];
+            const int32_t e = topk_idx[t * k + lane];
+            if (sl >= 0 && e >= 0 && e < E) {
+                row = offsets[e] + sl;
+                g = gates[t * k + lane];
+            }
+        }
+        int32_t rj[KMAX];
+        float gj[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            rj[j] = __shfl_sync(0xffffffffu, row, j);
+            gj[j] = __shfl_sync(0xffffffffu, g, j);
+        }
+        for (int c0 = 0; c0 < chunks; c0 += 32 * U) {
+            Raw raw[KMAX][U];
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (j < k && rj[j] >= 0 && c < chunks)
+                        raw[j][u] = Vec<T, VEC>::load_raw(out_rows + static_cast<int64_t>(rj[j]) * d + c * VEC);
+                }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c >= chunks) continue;
+                float acc[VEC];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) {
+                    if (j < k && rj[j] >= 0) {
+                        float o[VEC];
+                        Vec<T, VEC>::widen(raw[j][u], o);
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) acc[v] = fmaf(gj[j], o[v], acc[v]);
+                    }
+                }
+                Vec<T, VEC>::store(y + t * d + c * VEC, acc);
+            }
+        }
+    }
+}
+
+// MOE_COMBINE_WARP=0 keeps large batches on the per-chunk kernel (for comparisons).
+bool warp_combine_enabled() {
+    static const bool enabled = [] {
+        const char *v = getenv("MOE_COMBINE_WARP");
+        return v == nullptr || atoi(v) != 0;
+    }();
+    return enabled;
+}
+
 template <typename T, int VEC>
 cudaError_t launch_combine_t(const void *out_rows, const float *parts, int nparts,
                              int64_t part_stride, const int32_t *slot, const int32_t *topk_idx,
@@ -222,6 +301,25 @@ cudaError_t launch_combine_t(const void *out_rows, const float *parts, int npart
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int bpt = (chunks + 127) / 128;
+    if (N >= 2048 && nparts == 0 && VEC > 1 && k <= 8 && warp_combine_enabled()) {
+        int64_t blocks = (N + 7) / 8;  // 8 warps per block, one token per warp and pass
+        if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+        const unsigned gb = static_cast<unsigned>(blocks);
+        const T *o = static_cast<const T *>(out_rows);
+        T *yy = static_cast<T *>(y);
+        // KMAX * U = 6-8 loads of 16 bytes in flight per lane
+        if (k <= 2)
+            return launch_pdl(combine_warp_kernel<T, VEC, 2, 4>, dim3(gb), dim3(256), 0, s, o, slot, topk_idx,
+                              offsets, gates, N, d, k, E, yy);
+        if (k <= 4)
+            return launch_pdl(combine_warp_kernel<T, VEC, 4, 2>, dim3(gb), dim3(256), 0, s, o, slot, topk_idx,
+                              offsets, gates, N, d, k, E, yy);
+        if (k <= 6)
+            return launch_pdl(combine_warp_kernel<T, VEC, 6, 1>, dim3(gb), dim3(256), 0, s, o, slot, topk_idx,
+                              offsets, gates, N, d, k, E, yy);
+        return launch_pdl(combine_warp_kernel<T, VEC, 8, 1>, dim3(gb), dim3(256), 0, s, o, slot, topk_idx, offsets,
+                          gates, N, d, k, E, yy);
+    }
     if (N >= 2048 && nparts == 0 && N * bpt <= INT32_MAX) {
         return launch_pdl(combine_token_kernel<T, VEC>, dim3(static_cast<unsigned>(N * bpt)), dim3(128), 0, s,
                           static_cast<const T *>(out_rows), slot, topk_idx, offsets, gates, N, d, k, E, bpt,

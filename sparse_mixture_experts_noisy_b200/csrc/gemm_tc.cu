@@ -324,8 +324,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
             const Unit t = decode_unit<BN, SWAP>(u, pre_s, cnt_s, E, Nw, splits, kb_total);
             const int acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
-            const bool mine = mbar_wait_bounded(tfull0 + 8 * acc, acc_phase, status, tmo, 4);
-            if (!__all_sync(0xffffffffu, mine)) break;
+            if (!mbar_wait_warp(tfull0 + 8 * acc, acc_phase, status, tmo, 4)) break;
             tc_fence_after();
             const int cnt = cnt_s[t.e];
             const int64_t row_base = args.offsets[t.e];
@@ -607,8 +606,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
             decode(u, e, tok0, w0, kb0, kb1, nv);
             const int acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
-            const bool mine = mbar_wait_bounded(tfull0 + 8 * acc, acc_phase, status, tmo, 14);
-            if (!__all_sync(0xffffffffu, mine)) break;
+            if (!mbar_wait_warp(tfull0 + 8 * acc, acc_phase, status, tmo, 14)) break;
             tc_fence_after();
             const int cnt = cnt_s[e];
             const int my_row = tok0 + static_cast<int>(rank) * 128 + row_in_tile;

@@ -493,7 +493,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 14)) {
+                if (!mbar_wait_warp(xfull0 + 8 * stage, phase, status, tmo, 14)) {
                     ok = false;
                     break;
                 }
@@ -508,8 +508,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
         }
         // accumulator complete (every MMA, so every read of the ring, is done)
-        ok = ok && mbar_wait_bounded(accf, 0, status, tmo, 15);
         ok = __all_sync(0xffffffffu, ok);
+        ok = ok && mbar_wait_warp(accf, 0, status, tmo, 15);
         tc_fence_after();
         if (ok) {
             // this piece's sum per (token, expert) into the table [128][ld]
@@ -757,7 +757,7 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             bool ok = true;
             for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
                 for (int kb = 0; kb < kb_total; ++kb) {
-                    if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 25)) {
+                    if (!mbar_wait_warp(xfull0 + 8 * stage, phase, status, tmo, 25)) {
                         ok = false;
                         break;
                     }
@@ -786,8 +786,8 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             for (int c = 0; c < S; ++c, ++piece) {
                 const int b = piece & 1;
                 const uint32_t use = static_cast<uint32_t>(piece >> 1);
-                if (ok) ok = mbar_wait_bounded(accf0 + 8 * b, use & 1u, status, tmo, 26);
                 ok = __all_sync(0xffffffffu, ok);
+                if (ok) ok = mbar_wait_warp(accf0 + 8 * b, use & 1u, status, tmo, 26);
                 tc_fence_after();
                 if (ok) drain_piece<UPT>(tmem_base + lane_off + static_cast<uint32_t>(b * NB), c == 0, run);
                 tc_fence_before();
