@@ -385,3 +385,61 @@ class GraphedForward:
     def replay(self):
         self.graph.replay()
         return self.y
+
+
+class HostPipeline:
+    """The layer over a stream of batches that live in (pinned) host memory.
+
+    Two graphed forwards over two sets of device buffers alternate.  Batch i's
+    inputs are copied in on one stream, its forward replays on the current
+    stream, and its output is copied out on a third, with events between them,
+    so the copy of batch i+1 in and of batch i-1 out overlap the forward of
+    batch i.  `submit(x_h, y_h, noise_h)` enqueues one batch (x_h, noise_h
+    pinned host inputs, y_h the pinned host output); `synchronize()` waits for
+    all of them.  Host buffers must stay untouched until their batch is done."""
+
+    def __init__(self, layer: MoELayer, x_example, noise_example=None):
+        dev = x_example.device
+        self.graphs = []
+        for _ in range(2):
+            xb = torch.empty_like(x_example)
+            nb = None if noise_example is None else torch.empty_like(noise_example)
+            if nb is not None:
+                nb.copy_(noise_example)
+            xb.copy_(x_example)
+            self.graphs.append(GraphedForward(layer, xb, nb))
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.h2d = [torch.cuda.Event() for _ in range(2)]
+        self.done = [torch.cuda.Event() for _ in range(2)]
+        self.d2h = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+        self.i = 0
+
+    def submit(self, x_h, y_h, noise_h=None):
+        b = self.i & 1
+        g = self.graphs[b]
+        comp = torch.cuda.current_stream()
+        with torch.cuda.stream(self.s_in):
+            if self.used[b]:
+                self.s_in.wait_event(self.done[b])   # the forward of batch i-2 has read these inputs
+            g.x.copy_(x_h, non_blocking=True)
+            if noise_h is not None:
+                g.noise.copy_(noise_h, non_blocking=True)
+            self.h2d[b].record(self.s_in)
+        comp.wait_event(self.h2d[b])
+        if self.used[b]:
+            comp.wait_event(self.d2h[b])             # batch i-2's output has left these buffers
+        g.replay()
+        self.done[b].record(comp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.done[b])
+            y_h.copy_(g.y, non_blocking=True)
+            self.d2h[b].record(self.s_out)
+        self.used[b] = True
+        self.i += 1
+
+    def synchronize(self):
+        for b in range(2):
+            if self.used[b]:
+                self.d2h[b].synchronize()

@@ -184,3 +184,26 @@ def test_graph_replay_matches_eager_and_follows_new_inputs():
         y_ref = layer(other.x, noise=other.noise)
         torch.cuda.synchronize()
         assert torch.equal(y_new.view(torch.int16), y_ref.view(torch.int16))
+
+
+def test_host_pipeline_matches_eager():
+    """HostPipeline (two graphed forwards, copies in and out overlapping the
+    compute of neighbouring batches) returns each host batch's eager result
+    bit for bit, in order."""
+    wl = SMALL["mixtral_small"]
+    cases = [Case(wl, seed=s) for s in (11, 12, 13, 14, 15)]
+    layer = moe.MoELayer(cases[0].W_g, cases[0].W_up, cases[0].W_down, wl.k, wl.cf, b_g=cases[0].b_g,
+                         sigma=wl.sigma)
+    hosts = []
+    for c in cases:
+        xh = c.x.cpu().pin_memory()
+        nh = None if c.noise is None else c.noise.cpu().pin_memory()
+        hosts.append((xh, nh, torch.empty(xh.shape, dtype=xh.dtype).pin_memory()))
+    pipe = moe.HostPipeline(layer, cases[0].x, cases[0].noise)
+    for xh, nh, yh in hosts:
+        pipe.submit(xh, yh, nh)
+    pipe.synchronize()
+    for c, (_, _, yh) in zip(cases, hosts):
+        y_ref = layer(c.x, noise=c.noise)
+        torch.cuda.synchronize()
+        assert torch.equal(yh.view(torch.int16), y_ref.cpu().view(torch.int16))
