@@ -23,6 +23,8 @@ SMALL = {
     "nano_small": W["nano"].with_(N=1000, d=256, d_ff=384, wg_std=1 / 16),
     # router bias +1 on expert 0 overflows its capacity: drops
     "mixtral_small": W["mixtral"].with_(N=1536, d=512, d_ff=1024),
+    # ragged N in both projections (720 = 2 * 256 + 208, 640 = 2 * 256 + 128)
+    "ragged_pair": W["mixtral"].with_(N=1536, d=640, d_ff=720),
     # 64 experts, k = 6, supplied noise, d_ff not a multiple of the N tile
     "fine_small": W["fine"].with_(N=2048, d=256, d_ff=176),
     # few tokens per expert: weight-stationary tiles and split-K down projection
