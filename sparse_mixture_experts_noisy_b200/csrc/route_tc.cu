@@ -311,27 +311,45 @@ __device__ __forceinline__ void pick_row_smem(const float *sr, int E, int k, flo
     for (int j = 0; j < k; ++j) gt[j] = __fdiv_rn(expf(__fsub_rn(pv_s[j], mx)), sum);
 }
 
-// The same for scores held in registers (s[0..E), E <= E_PAD).
+// The same for scores held in registers (s[0..E), E <= E_PAD; s is consumed).
+// Each score becomes a 64-bit key whose order is the pick order: high word
+// the score mapped to an unsigned that orders like the float (-0 taken as +0,
+// so equal floats give equal words), low word ~e (lower index ranks first on
+// ties).  A round takes the largest key below the previous pick, as 8
+// independent running maxima folded at the end.
+__device__ __forceinline__ uint32_t ordered_bits(float v) {
+    const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered_bits(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 template <int E_PAD>
-__device__ __forceinline__ void pick_row_regs(const float (&s)[E_PAD], int E, int k, float *pv_s, int32_t *ti,
+__device__ __forceinline__ void pick_row_regs(float (&s)[E_PAD], int E, int k, float *pv_s, int32_t *ti,
                                               float *gt) {
-    float pv = 0.0f;
-    int pe = -1;
+    uint32_t u[E_PAD];
+#pragma unroll
+    for (int e = 0; e < E_PAD; ++e) u[e] = ordered_bits(s[e]);
+    uint64_t prev = ~0ull;  // the first round takes the largest key
     for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int be = -1;
+        uint64_t part[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[i] = 0;
 #pragma unroll
         for (int e = 0; e < E_PAD; ++e) {
-            if (e < E && (pe < 0 || ranks_before_tc(pv, pe, s[e], e)) &&
-                (be < 0 || ranks_before_tc(s[e], e, bv, be))) {
-                bv = s[e];
-                be = e;
-            }
+            const uint64_t key = (static_cast<uint64_t>(u[e]) << 32) | static_cast<uint32_t>(~e);
+            const uint64_t cand = (e < E && key < prev) ? key : 0ull;
+            part[e & 7] = cand > part[e & 7] ? cand : part[e & 7];
         }
-        ti[j] = be;
-        pv_s[j] = bv;
-        pv = bv;
-        pe = be;
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) part[i] = part[i + w] > part[i] ? part[i + w] : part[i];
+        const uint64_t best = part[0];
+        ti[j] = static_cast<int32_t>(~static_cast<uint32_t>(best));
+        pv_s[j] = from_ordered_bits(static_cast<uint32_t>(best >> 32));
+        prev = best;
     }
     const float mx = pv_s[0];
     float sum = 0.0f;
