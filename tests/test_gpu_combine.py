@@ -17,7 +17,7 @@ from tests.gpu_util import require_gpu
 pytestmark = pytest.mark.gpu
 
 
-def _case(k, N=2100, d=520, E=9, cf=0.9, seed=0):
+def _case(k, N=2100, d=520, E=12, cf=0.9, seed=0):
     rng = np.random.default_rng(100 + k)
     scores = rng.standard_normal((N, E))
     topk = np.argsort(-scores, axis=1, kind="stable")[:, :k].astype(np.int32)
@@ -31,10 +31,13 @@ def _case(k, N=2100, d=520, E=9, cf=0.9, seed=0):
     return tk, torch.from_numpy(g).cuda(), disp, out_t, out
 
 
-@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 6, 7, 8])
-def test_combine_variants(k):
+@pytest.mark.parametrize("k,d", [(1, 520), (2, 520), (3, 520), (4, 520), (5, 520), (6, 520), (7, 520), (8, 520),
+                                 (10, 520), (2, 36)])
+def test_combine_variants(k, d):
+    """k <= 8 with 16-byte rows: the warp kernel; k = 10 or d = 36 (rows not
+    16-byte multiples): the per-chunk kernel."""
     require_gpu()
-    tk, g, disp, out_t, out = _case(k)
+    tk, g, disp, out_t, out = _case(k, d=d)
     y = moe.moe_combine(out_t, disp["slot"], tk, disp["offsets"], g)
     torch.cuda.synchronize()
     yb = y.view(torch.int16).cpu().numpy().view(np.uint16)
