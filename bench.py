@@ -481,9 +481,10 @@ def run_ours(args):
                                         "whole_layer_gbs": layer_bytes / (dmax / dsteps) / 1e9,
                                         "whole_layer_frac": layer_bytes / (dmax / dsteps) / 1e9 / peaks["hbm_gbs"],
                                         "whole_layer_frac_of_8tbs": layer_bytes / (dmax / dsteps) / 8e12}),
-            "clocks": dclk}
-        line["gpu_launches"] += moe.forward_launches(dwl.N, dwl.d, dwl.E, dwl.d_ff, dwl.k, dwl.cf,
-                                                     ddev[0].dtype) * dsteps
+            "clocks": dclk,
+            # the decode run's own timed region (the top-level count is the main one's)
+            "gpu_launches": moe.forward_launches(dwl.N, dwl.d, dwl.E, dwl.d_ff, dwl.k, dwl.cf,
+                                                 ddev[0].dtype) * dsteps}
 
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cores = cpu_cores()
