@@ -153,6 +153,37 @@ void oracle_assign_slots(const int32_t *topk_idx, int64_t N, int E, int k, int64
     free(queue);
 }
 
+/* Per-expert load of one routed batch ("nanoMoEの深層解剖" slide 14: the
+ * router's used_capacity counts each expert's rows that survive the capacity
+ * cut).  load[e]: choices (t, j) that picked e, before the cut; used[e] =
+ * min(load[e], C); importance[e] (skipped if gates or importance is NULL):
+ * the sum of those choices' gates, each gate taken as the nearest multiple of
+ * 2^-32 (ties to even), summed exactly in 64-bit integers, then scaled back. */
+void oracle_load_stats(const int32_t *topk_idx, const float *gates, int64_t N, int E, int k, int64_t C,
+                       int32_t *load, int32_t *used, double *importance)
+{
+    int64_t *q = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *mass = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    for (int64_t t = 0; t < N; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = topk_idx[(size_t)t * k + j];
+            if (e < 0 || e >= E)
+                continue;
+            q[e] += 1;
+            if (gates)
+                mass[e] += llrint(ldexp((double)gates[(size_t)t * k + j], 32));
+        }
+    }
+    for (int e = 0; e < E; ++e) {
+        load[e] = (int32_t)q[e];
+        used[e] = (int32_t)(q[e] < C ? q[e] : C);
+        if (gates && importance)
+            importance[e] = ldexp((double)mass[e], -32);
+    }
+    free(q);
+    free(mass);
+}
+
 /* The nanoMoE expert variant ("nanoMoEの深層解剖" slide 32, MLPExperts): an
  * optional bias after each projection and GELU in place of ReLU.  GELU is the
  * exact form x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2)), in double.

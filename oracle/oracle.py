@@ -50,6 +50,8 @@ def _load():
             lib.oracle_capacity.restype = I64
             lib.oracle_assign_slots.argtypes = [P, I64, I32, I32, I64, P, P]
             lib.oracle_assign_slots.restype = None
+            lib.oracle_load_stats.argtypes = [P, P, I64, I32, I32, I64, P, P, P]
+            lib.oracle_load_stats.restype = None
             lib.oracle_expert_ffn.argtypes = [P, I32, P, P, I64, I32, I32, I32, P, P]
             lib.oracle_expert_ffn.restype = None
             lib.oracle_ffn_combine.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, P, I64, P, I32]
@@ -111,6 +113,20 @@ def assign_slots(topk_idx, E, C):
     counts = np.empty(E, dtype=np.int32)
     _load().oracle_assign_slots(_ptr(topk_idx), N, E, k, int(C), _ptr(slot), _ptr(counts))
     return slot, counts
+
+
+def load_stats(topk_idx, E, C, gates=None):
+    """(load [E] int32, used [E] int32, importance [E] float64 or None): per-expert
+    choices before the capacity cut, min(load, C) (slide 14's used_capacity),
+    and the gate mass in units of 2^-32 summed exactly."""
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    N, k = topk_idx.shape
+    load = np.empty(E, dtype=np.int32)
+    used = np.empty(E, dtype=np.int32)
+    imp = np.empty(E, dtype=np.float64) if gates is not None else None
+    g = None if gates is None else np.ascontiguousarray(gates, dtype=np.float32)
+    _load().oracle_load_stats(_ptr(topk_idx), _ptr(g), N, E, k, int(C), _ptr(load), _ptr(used), _ptr(imp))
+    return load, used, imp
 
 
 def expert_ffn(x, W_up, W_down, t, e):

@@ -363,8 +363,57 @@ def check_gelu_bias_layer(seed=13):
     np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
 
 
+def check_load_stats_m2():
+    """Slide 14's used_capacity on the capacity example (slides 15-23): used =
+    1, 1, 1 at capacity 1; the load before the cut is one more than each
+    expert's last queue place in the uncut ranking (slides 18-19); the gate
+    mass is the sum of slide 24's picked probabilities per expert."""
+    m2 = load_m2()
+    topk = np.array(m2["topk"], dtype=np.int32)
+    gates = np.array(m2["gates"], dtype=np.float32)
+    load, used, imp = oracle.load_stats(topk, m2["E"], m2["C"], gates)
+    assert used.tolist() == m2["used"], used.tolist()
+    rank = np.array(m2["rank_nocap"])
+    expect_load = [int(rank[topk == e].max()) + 1 for e in range(m2["E"])]
+    assert load.tolist() == expect_load, (load.tolist(), expect_load)
+    g64 = np.array(m2["gates"], dtype=np.float32).astype(np.float64)
+    for e in range(m2["E"]):
+        mass = float(g64[topk == e].sum())
+        assert abs(imp[e] - mass) <= (topk == e).sum() * 2.0 ** -33, (e, imp[e], mass)
+
+
+def check_load_stats_random(seed=14):
+    """On random routings: load is numpy's bincount of the choices; used is
+    the slot pass's per-expert count and min(load, C); the gate mass is within
+    one 2^-33 rounding per choice of numpy's float64 weighted bincount, and
+    exact when every gate is a multiple of 2^-32."""
+    rng = np.random.default_rng(seed)
+    for N, E, k, cf in ((500, 8, 2, 0.7), (257, 13, 3, 1.0), (64, 64, 6, math.inf)):
+        topk = np.stack([rng.permutation(E)[:k] for _ in range(N)]).astype(np.int32)
+        gates = rng.random((N, k)).astype(np.float32)
+        C = oracle.capacity(N, E, k, cf)
+        load, used, imp = oracle.load_stats(topk, E, C, gates)
+        assert np.array_equal(load, np.bincount(topk.ravel(), minlength=E))
+        _, counts = oracle.assign_slots(topk, E, C)
+        assert np.array_equal(used, counts)
+        assert np.array_equal(used, np.minimum(load, C))
+        ref = np.bincount(topk.ravel(), weights=gates.ravel().astype(np.float64), minlength=E)
+        assert np.all(np.abs(imp - ref) <= load * 2.0 ** -33 + 1e-300)
+        dyadic = (np.floor(gates.astype(np.float64) * 64.0) / 64.0).astype(np.float32)
+        _, _, imp2 = oracle.load_stats(topk, E, C, dyadic)
+        ref2 = np.bincount(topk.ravel(), weights=dyadic.ravel().astype(np.float64), minlength=E)
+        assert np.array_equal(imp2, ref2)
+    # the rounding of each gate to units of 2^-32 is to nearest, ties to even:
+    # 0.75 -> 1, 0.5 -> 0, 1.5 -> 2, 2.5 -> 2 units
+    u = 2.0 ** -32
+    topk = np.zeros((4, 1), dtype=np.int32)
+    gates = np.array([[0.75 * u], [0.5 * u], [1.5 * u], [2.5 * u]], dtype=np.float32)
+    _, _, imp = oracle.load_stats(topk, 1, 4, gates)
+    assert imp[0] == 5 * u, imp[0] / u
+
+
 ALL_CHECKS = [check_m1, check_m2_slots, check_m2_combine, check_topk_bruteforce,
               check_gates_invariants, check_noise, check_capacity, check_slots_bruteforce,
               check_logits_vs_numpy, check_ffn_vs_numpy, check_dense_mixture,
               check_single_expert_mlp, check_all_dropped_is_zero, check_gelu_expert_variant,
-              check_gelu_bias_layer]
+              check_gelu_bias_layer, check_load_stats_m2, check_load_stats_random]

@@ -44,6 +44,10 @@ MUTANTS = {
     "down_bias_dropped": ("acc += (double)b_down[(size_t)e * d + i];", "acc += 0.0 * b_down[(size_t)e * d + i];"),
     "softmax_not_shifted_sign": ("denom += exp((double)s[idx[j]] - top);",
                                  "denom += exp(top - (double)s[idx[j]]);"),
+    "used_not_capped": ("used[e] = (int32_t)(q[e] < C ? q[e] : C);", "used[e] = (int32_t)q[e];"),
+    "load_counts_once_per_token": ("            q[e] += 1;\n", "            q[e] += (j == 0);\n"),
+    "gate_mass_truncated": ("mass[e] += llrint(ldexp((double)gates[(size_t)t * k + j], 32));",
+                            "mass[e] += (int64_t)ldexp((double)gates[(size_t)t * k + j], 32);"),
 }
 
 
@@ -68,7 +72,7 @@ def test_pins_catch_mutant(tmp_path, name):
         mutant = ctypes.CDLL(lib_path)
         for fn in ("oracle_router_logits", "oracle_route_from_logits", "oracle_capacity",
                    "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine",
-                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex"):
+                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex", "oracle_load_stats"):
             getattr(mutant, fn).argtypes = getattr(saved, fn).argtypes
             getattr(mutant, fn).restype = getattr(saved, fn).restype
         O._lib = mutant
