@@ -242,6 +242,27 @@ MOE_API moe_status moe_combine(const void *out_gathered, const int32_t *slot, co
                        const int32_t *offsets, const float *gates, moe_dtype dt, int64_t N,
                        int d, int k, void *y, void *stream);
 
+/* ---------------------------------------------------------------- load statistics */
+
+/* Per-expert load of one routed batch ("nanoMoEの深層解剖" slide 14: the
+ * router's used_capacity counts each expert's rows that survive the capacity
+ * cut; STEP 4's noise exists to spread this load).  No gradient or loss form
+ * is on the pages; these are the quantities a balancing loss would use.
+ *  topk_idx   device [N, k] int32 (from moe_route); entries outside [0, E) are skipped
+ *  gates      device [N, k] fp32 or NULL
+ *  cf         capacity factor, as for moe_dispatch (C = moe_capacity(N, E, k, cf))
+ *  load       device [E] int32 out: choices (t, j) that picked e, before the cut
+ *  used       device [E] int32 out: min(load[e], C), equal to moe_dispatch's counts
+ *  importance device [E] double out or NULL: the gates of load's choices summed,
+ *             each gate rounded to the nearest multiple of 2^-32 (ties to even) and
+ *             added exactly, so the result does not depend on the order of the adds
+ *  ws, ws_bytes  workspace of at least moe_load_stats_workspace_size() bytes
+ * E <= 256, N * k < 2^31.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_WORKSPACE, MOE_ERR_CUDA. */
+MOE_API size_t moe_load_stats_workspace_size(void);
+MOE_API moe_status moe_load_stats(const int32_t *topk_idx, const float *gates, int64_t N, int E, int k,
+                                  double cf, int32_t *load, int32_t *used, double *importance, void *ws,
+                                  size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- fused */
 
 /* Workspace bytes for moe_forward. */

@@ -399,6 +399,31 @@ moe_status moe_combine(const void *out_gathered, const int32_t *slot, const int3
     return MOE_OK;
 }
 
+size_t moe_load_stats_workspace_size(void) { return moe::stats_ws_bytes(); }
+
+moe_status moe_load_stats(const int32_t *topk_idx, const float *gates, int64_t N, int E, int k, double cf,
+                          int32_t *load, int32_t *used, double *importance, void *ws, size_t ws_bytes,
+                          void *stream) {
+    if (N < 0 || E < 1 || E > moe::kStatsMaxE || k < 1 || k > E)
+        return fail(MOE_ERR_INVALID_ARG, "need N >= 0 and 1 <= k <= E <= %d", moe::kStatsMaxE);
+    if (N * static_cast<int64_t>(k) >= (static_cast<int64_t>(1) << 31))
+        return fail(MOE_ERR_INVALID_ARG, "N * k must be below 2^31");
+    const int64_t C = moe_capacity(N, E, k, cf);
+    if (C < 0) return fail(MOE_ERR_INVALID_ARG, "capacity factor must be > 0 or +inf (got %g)", cf);
+    if (N > 0) REQUIRE_PTR(topk_idx, "topk_idx");
+    OPTIONAL_PTR(gates, "gates");
+    REQUIRE_PTR(load, "load");
+    REQUIRE_PTR(used, "used");
+    OPTIONAL_PTR(importance, "importance");
+    if (ws == nullptr || ws_bytes < moe::stats_ws_bytes())
+        return fail(MOE_ERR_WORKSPACE, "load statistics need %zu bytes of workspace", moe::stats_ws_bytes());
+    REQUIRE_PTR(ws, "ws");
+    cudaError_t e = moe::launch_load_stats(topk_idx, gates, N, E, k, C, load, used, importance, ws,
+                                           static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "load statistics launch");
+    return MOE_OK;
+}
+
 size_t moe_workspace_size(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt) {
     if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1) return 0;
     const int64_t C = moe_capacity(N, E, k, cf);

@@ -72,6 +72,13 @@ cudaError_t launch_gather(const int32_t *topk_idx, const int32_t *slot, const in
                           const void *x, int elem_bytes, int64_t N, int d, int k, void *x_gathered,
                           cudaStream_t s);
 
+// Per-expert load statistics (stats.cu): load before the capacity cut, used =
+// min(load, C), gate mass in exact units of 2^-32.  E <= kStatsMaxE.
+constexpr int kStatsMaxE = 256;
+size_t stats_ws_bytes();
+cudaError_t launch_load_stats(const int32_t *topk_idx, const float *gates, int64_t N, int E, int k, int64_t C,
+                              int32_t *load, int32_t *used, double *importance, void *ws, cudaStream_t s);
+
 // Combine (combine.cu).  Either out_rows (dtype rows, nparts == 0) or nparts
 // fp32 partial buffers `part_stride` elements apart.
 // b_down (nullable, [E][d]) is added to the summed partials (nparts > 0 only;

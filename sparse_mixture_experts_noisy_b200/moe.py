@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_shard_workspace_size", "moe_shard_count", "moe_shard_base", "moe_shard_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_combine",
+           "moe_load_stats_workspace_size", "moe_load_stats",
            "moe_workspace_size", "moe_forward", "moe_forward_ex", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
 
@@ -56,6 +57,8 @@ def load_library(path: str = LIB_PATH):
             "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
             "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
             "moe_dispatch_noalloc": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P]),
+            "moe_load_stats_workspace_size": (SZ, []),
+            "moe_load_stats": (I, [P, P, I64, I, I, D, P, P, P, P, SZ, P]),
             "moe_shard_workspace_size": (SZ, [I64, I, I]),
             "moe_shard_count": (I, [P, I64, I, I, P, P, SZ, P]),
             "moe_shard_base": (I, [P, I, I, I, I, P, P]),
@@ -267,6 +270,23 @@ def moe_combine(out_gathered, slot, topk_idx, offsets, gates, stream=None, y=Non
     _check(L.moe_combine(_p(out_gathered), _p(slot), _p(topk_idx), _p(offsets), _p(gates),
                          _dt(out_gathered), N, d, k, _p(y), _stream(stream)))
     return y
+
+
+def moe_load_stats(topk_idx, E, cf, gates=None, stream=None):
+    """Per-expert load of a routed batch (slide 14's used_capacity and more).
+    -> dict(load [E] int32, used [E] int32, importance [E] float64 or None)."""
+    L = load_library()
+    _cuda(topk_idx, "topk_idx")
+    _cuda(gates, "gates")
+    N, k = topk_idx.shape
+    dev = topk_idx.device
+    load = torch.empty(E, dtype=torch.int32, device=dev)
+    used = torch.empty(E, dtype=torch.int32, device=dev)
+    imp = torch.empty(E, dtype=torch.float64, device=dev) if gates is not None else None
+    ws = torch.empty(max(int(L.moe_load_stats_workspace_size()), 256), dtype=torch.uint8, device=dev)
+    _check(L.moe_load_stats(_p(topk_idx), _p(gates), N, E, k, _cf(cf), _p(load), _p(used), _p(imp), _p(ws),
+                            ws.numel(), _stream(stream)))
+    return dict(load=load, used=used, importance=imp)
 
 
 def workspace_size(N, d, E, d_ff, k, cf, dtype) -> int:

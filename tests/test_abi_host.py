@@ -105,6 +105,21 @@ def test_expert_ffn_and_forward_reject_bad_arguments(L):
     assert L.moe_debug_wait_timeout(0, a, 4096, None) == 1
 
 
+def test_load_stats_rejects_bad_arguments(L):
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    ws = int(L.moe_load_stats_workspace_size())
+    assert ws >= 256 * 12
+    assert L.moe_load_stats(a, None, 16, 300, 2, 1.0, a, a, None, a, ws, None) == 1   # E > 256
+    assert L.moe_load_stats(a, None, 16, 4, 5, 1.0, a, a, None, a, ws, None) == 1     # k > E
+    assert L.moe_load_stats(a, None, 16, 4, 2, 0.0, a, a, None, a, ws, None) == 1     # cf
+    assert "capacity factor" in _err(L)
+    assert L.moe_load_stats(a, None, 16, 4, 2, 1.0, None, a, None, a, ws, None) == 1  # load NULL
+    assert L.moe_load_stats(a, P(0x10004), 16, 4, 2, 1.0, a, a, None, a, ws, None) == 1  # misaligned gates
+    assert L.moe_load_stats(a, None, 16, 4, 2, 1.0, a, a, None, a, 8, None) == 3       # workspace
+    assert "workspace" in _err(L)
+
+
 def test_workspace_sizes_are_monotone(L):
     s1 = L.moe_workspace_size(1024, 256, 8, 512, 2, 1.25, 1)
     s2 = L.moe_workspace_size(2048, 256, 8, 512, 2, 1.25, 1)
