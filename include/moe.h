@@ -95,12 +95,12 @@ MOE_API int64_t moe_gathered_rows(int64_t N, int E, int k, double cf);
  *  logits_out device [N, E] fp32 or NULL    receives s_raw (bias included, before noise)
  *  topk_idx   device [N, k] int32           kept experts, first choice first
  *  gates      device [N, k] fp32            softmax of the kept scores, same order
- * The dot products accumulate in fp32.  bf16 batches of more than 1024 tokens
- * (d a multiple of 8, x and W_g 16-byte aligned, E <= 160) run them on the
- * tensor cores with each fp32 weight split exactly into three bf16 parts, so
- * every product is exact and only the fp32 accumulation rounds; other shapes
- * run on CUDA cores.  Either way the top-k and softmax are the same given the
- * logits. */
+ * The dot products accumulate in fp32.  bf16 tokens (d a multiple of 8,
+ * E <= 160, k <= 32) run them on the tensor cores with each fp32 weight split
+ * exactly into three bf16 parts, so every product is exact and only the fp32
+ * accumulation rounds; other shapes run on CUDA cores.  Either way the top-k
+ * and softmax are the same given the logits, and a token's results do not
+ * depend on N or on its position in the batch. */
 MOE_API moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                      const float *noise, float sigma, int64_t N, int d, int E, int k,
                      float *logits_out, int32_t *topk_idx, float *gates, void *stream);

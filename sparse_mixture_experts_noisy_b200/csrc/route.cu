@@ -5,7 +5,7 @@
 // "nanoMoEの深層解剖" slides 11-13 (router in fp32 with autocast disabled, topk,
 // -inf scatter, softmax).
 //
-// bf16 tokens with d a multiple of 8 and at most 160 experts route on the
+// bf16 tokens with d a multiple of 8, at most 160 experts and k <= 32 route on the
 // tensor cores (route_tc.cu).  Everything else runs here, on CUDA cores in
 // fp32 (fmaf), in one of two launch shapes: large batches give 4 tokens to
 // each warp with W_g staged in shared memory, small batches give one token to
