@@ -16,7 +16,9 @@
  *     slides 12-13 (topk, -inf scatter, softmax), slide 14 and slides 15-23
  *     (one_hot + cumsum slot rank with all first choices ranked before all
  *     second choices, capacity drop), slides 24-29 and 38-40 (combine with
- *     the pre-drop gate, dropped pairs contribute nothing).
+ *     the pre-drop gate, dropped pairs contribute nothing), slide 32 (the
+ *     MLPExperts variant: biases, GELU), slide 14 (used_capacity, extended to
+ *     per-expert load statistics).
  *
  * Readings where the pages leave a step open:
  *   - noise: s = fl32(s_raw + fl32(sigma * eps)) with eps ~ N(0,1) supplied;
