@@ -6,6 +6,9 @@
    choices of e, dropped at the whole batch's capacity).  Rank 0 checks the
    union against the unsharded oracle.
 2. bench.py's rank plumbing: max over ranks and whole-job throughput.
+3. Expert parallelism: every rank's exchange plan (rows it sends to and
+   receives from each rank) agrees with every other rank's, and ep.Comm's
+   all-to-all delivers each block to its owner and back.
 """
 import datetime
 import math
@@ -103,3 +106,50 @@ def _bench_worker(rank, world, port):
 
 def test_bench_takes_the_slowest_rank():
     mp.start_processes(_bench_worker, args=(2, _port()), nprocs=2, start_method="spawn", join=True)
+
+
+def _ep_worker(rank, world, port, E, seed):
+    import sys
+    sys.path.insert(0, ROOT)
+    from sparse_mixture_experts_noisy_b200 import ep
+    _init(rank, world, port)
+    try:
+        comm = ep.Comm()
+        rng = np.random.default_rng(seed + rank)
+        kept = torch.from_numpy(rng.integers(0, 9, size=E).astype(np.int32))
+        kept_all = comm.all_gather(kept)
+        assert kept_all.shape == (world, E) and torch.equal(kept_all[rank], kept)
+        plan = ep.ep_plan(kept_all.tolist(), world, rank)
+        plans = [None] * world
+        dist.all_gather_object(plans, (plan.send_splits, plan.recv_splits, plan.recv_counts))
+        for q in range(world):
+            assert plans[q][0][rank] == plan.recv_splits[q]
+            lo, hi = ep.expert_range(E, world, rank)
+            assert plan.recv_counts[q] == kept_all[q, lo:hi].tolist()
+        # rows tagged (source, expert, row) travel to the expert's owner and back
+        d = 3
+        rows = []
+        for e in range(E):
+            for i in range(int(kept[e])):
+                rows.append([rank, e, i])
+        xg = torch.tensor(rows, dtype=torch.float32).reshape(-1, d)
+        sends = [xg[s0:s0 + n] for s0, n in zip(plan.send_offsets, plan.send_splits)]
+        recv = [torch.empty((n, d)) for n in plan.recv_splits]
+        comm.all_to_all(recv, sends)
+        lo, hi = ep.expert_range(E, world, rank)
+        for s in range(world):
+            got = recv[s]
+            assert torch.all(got[:, 0] == s)
+            assert torch.all((got[:, 1] >= lo) & (got[:, 1] < hi))
+            assert got.shape[0] == sum(plan.recv_counts[s])
+        back = [torch.empty_like(t) for t in sends]
+        comm.all_to_all(back, [r.clone() for r in recv])
+        assert torch.equal(torch.cat(back), xg)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E", [(2, 8), (4, 8), (3, 7)])
+def test_expert_parallel_exchange(world, E):
+    mp.start_processes(_ep_worker, args=(world, _port(), E, 21), nprocs=world, start_method="spawn", join=True)
