@@ -155,6 +155,105 @@ void oracle_assign_slots(const int32_t *topk_idx, int64_t N, int E, int k, int64
     free(queue);
 }
 
+/* Backward of the layer for a given routing.  "Mixture of Experts (MoE)
+ * 12段階極小ビジュアル解剖シミュレーター" STEP 6 (the -inf mask keeps the kept
+ * experts' softmax differentiable and gives the others gate 0) and STEP 11
+ * (g_i E_i(x) carries the gradient to the router); the top-k indices and the
+ * slots are piecewise constant and carry none.  With L = sum over t, i of
+ * dy[t, i] y[t, i]:
+ *   kept (t, j), e = topk[t, j]:  z = W_up[e] x_t,  h = ReLU(z),  o = W_down[e] h
+ *     dg_j = dy_t . o,   d_o = g_j dy_t
+ *     dW_down[e] += d_o h^T,  dz = (W_down[e]^T d_o) * [z > 0],
+ *     dW_up[e] += dz x_t^T,   dx_t += W_up[e]^T dz
+ *   dropped (t, j): dg_j = 0 (its gate multiplies nothing)
+ *   every chosen (t, j): ds_j = g_j (dg_j - sum_l g_l dg_l)   (softmax over the k
+ *     chosen scores, capacity drops included, as the gates are formed before the cut)
+ *     db_g[e] += ds_j,  dW_g[e] += ds_j x_t,  dx_t += ds_j W_g[e]
+ * s [N, E] fp32 are the noisy scores the gates came from (s = s_raw + sigma eps:
+ * ds_raw = ds); the gates are recomputed from them in double.  dy [N, d] double.
+ * Outputs are double and overwritten: dx [N, d], dW_g [E, d], db_g [E],
+ * dW_up [E, d_ff, d], dW_down [E, d, d_ff]. */
+void oracle_backward(const void *x, int dt, const float *W_g, const void *W_up, const void *W_down,
+                     const float *s, const int32_t *topk_idx, const int32_t *slot, const double *dy,
+                     int64_t N, int d, int E, int d_ff, int k,
+                     double *dx, double *dW_g, double *db_g, double *dW_up, double *dW_down)
+{
+    memset(dx, 0, sizeof(double) * (size_t)N * d);
+    memset(dW_g, 0, sizeof(double) * (size_t)E * d);
+    memset(db_g, 0, sizeof(double) * (size_t)E);
+    memset(dW_up, 0, sizeof(double) * (size_t)E * d_ff * d);
+    memset(dW_down, 0, sizeof(double) * (size_t)E * d * d_ff);
+    double *g = (double *)malloc(sizeof(double) * (size_t)k);
+    double *dg = (double *)malloc(sizeof(double) * (size_t)k);
+    double *z = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    double *h = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    double *dz = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int64_t t = 0; t < N; ++t) {
+        const int32_t *ti = topk_idx + (size_t)t * k;
+        const double top = (double)s[(size_t)t * E + ti[0]];
+        double denom = 0.0;
+        for (int j = 0; j < k; ++j)
+            denom += exp((double)s[(size_t)t * E + ti[j]] - top);
+        for (int j = 0; j < k; ++j)
+            g[j] = exp((double)s[(size_t)t * E + ti[j]] - top) / denom;
+        const double *dyt = dy + (size_t)t * d;
+        double *dxt = dx + (size_t)t * d;
+        for (int j = 0; j < k; ++j) {
+            dg[j] = 0.0;
+            if (slot[(size_t)t * k + j] < 0)
+                continue;
+            const int e = ti[j];
+            for (int f = 0; f < d_ff; ++f) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i)
+                    acc += elem(W_up, dt, ((size_t)e * d_ff + f) * d + i) * elem(x, dt, (size_t)t * d + i);
+                z[f] = acc;
+                h[f] = acc > 0.0 ? acc : 0.0;
+            }
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int f = 0; f < d_ff; ++f)
+                    acc += elem(W_down, dt, ((size_t)e * d + i) * d_ff + f) * h[f];
+                o[i] = acc;
+                dg[j] += dyt[i] * acc;
+            }
+            for (int f = 0; f < d_ff; ++f) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    const double d_o = g[j] * dyt[i];
+                    dW_down[((size_t)e * d + i) * d_ff + f] += d_o * h[f];
+                    acc += elem(W_down, dt, ((size_t)e * d + i) * d_ff + f) * d_o;
+                }
+                dz[f] = z[f] > 0.0 ? acc : 0.0;
+            }
+            for (int f = 0; f < d_ff; ++f)
+                for (int i = 0; i < d; ++i) {
+                    dW_up[((size_t)e * d_ff + f) * d + i] += dz[f] * elem(x, dt, (size_t)t * d + i);
+                    dxt[i] += elem(W_up, dt, ((size_t)e * d_ff + f) * d + i) * dz[f];
+                }
+        }
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j)
+            sum += g[j] * dg[j];
+        for (int j = 0; j < k; ++j) {
+            const double ds = g[j] * (dg[j] - sum);
+            const int e = ti[j];
+            db_g[e] += ds;
+            for (int i = 0; i < d; ++i) {
+                dW_g[(size_t)e * d + i] += ds * elem(x, dt, (size_t)t * d + i);
+                dxt[i] += ds * (double)W_g[(size_t)e * d + i];
+            }
+        }
+    }
+    free(g);
+    free(dg);
+    free(z);
+    free(h);
+    free(dz);
+    free(o);
+}
+
 /* Per-expert load of one routed batch ("nanoMoEの深層解剖" slide 14: the
  * router's used_capacity counts each expert's rows that survive the capacity
  * cut).  load[e]: choices (t, j) that picked e, before the cut; used[e] =

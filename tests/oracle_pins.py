@@ -7,7 +7,8 @@ build of the oracle) run the very same checks.
 Sources of truth used here, none of which is the oracle's own code:
   * the nanoMoE slides' worked examples (tests/golden/*.txt, with citations),
   * brute-force enumeration of expert subsets and of queue places,
-  * numpy/scipy float64 library routines (matmul, softmax),
+  * numpy/scipy float64 library routines (matmul, softmax) and torch's
+    float64 autograd (for the backward),
   * closed forms and invariants of the definition (gates sum to 1, sigma = 0
     leaves the scores unchanged, k = E with no capacity limit is the dense
     softmax mixture, E = 1 and k = 1 is a plain ReLU MLP).
@@ -412,8 +413,68 @@ def check_load_stats_random(seed=14):
     assert imp[0] == 5 * u, imp[0] / u
 
 
+def _autograd_grads(x64, Wg64, bg64, Wu64, Wd64, eps64, sigma, s32, topk, slot, dy):
+    """torch float64 autograd of L = sum(dy * y) with the routing held fixed;
+    the scores take the oracle's fp32 values s32 with an identity gradient."""
+    import torch
+    T = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)  # noqa: E731
+    X, G, B, U, D = T(x64), T(Wg64), T(bg64), T(Wu64), T(Wd64)
+    S = X @ G.T + B + sigma * torch.tensor(eps64, dtype=torch.float64)
+    S = S + (torch.tensor(s32.astype(np.float64)) - S).detach()
+    g = torch.softmax(S.gather(1, torch.tensor(topk, dtype=torch.int64)), dim=1)
+    N, k = topk.shape
+    rows = []
+    for t in range(N):
+        acc = torch.zeros(x64.shape[1], dtype=torch.float64)
+        for j in range(k):
+            if slot[t, j] >= 0:
+                e = int(topk[t, j])
+                acc = acc + g[t, j] * (D[e] @ torch.relu(U[e] @ X[t]))
+        rows.append(acc)
+    L = (torch.stack(rows) * torch.tensor(dy)).sum()
+    L.backward()
+    return dict(dx=X.grad.numpy(), dW_g=G.grad.numpy(), db_g=B.grad.numpy(), dW_up=U.grad.numpy(),
+                dW_down=D.grad.numpy())
+
+
+def check_backward_vs_autograd(seed=15):
+    """The backward (STEP 6: the masked softmax stays differentiable; STEP 11:
+    g_i E_i(x) carries the gradient to the router) against torch's float64
+    autograd of the same forward with the routing fixed: fp32 and bf16
+    storage, noise, bias, capacity drops (a dropped choice's score still
+    enters the softmax), and k = 1 (the router gets no gradient)."""
+    from sparse_mixture_experts_noisy_b200.synth import bf16_bits_to_f32, f32_to_bf16_bits
+    rng = np.random.default_rng(seed)
+    for N, d, E, d_ff, k, cf, sigma, bf16 in ((7, 5, 4, 6, 2, 0.6, 0.7, False), (9, 8, 6, 5, 3, 0.5, 0.0, True),
+                                              (5, 4, 3, 4, 1, 1.0, 0.3, False)):
+        x = rng.standard_normal((N, d)).astype(np.float32)
+        Wg = rng.standard_normal((E, d)).astype(np.float32)
+        bg = rng.standard_normal(E).astype(np.float32)
+        Wu = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+        Wd = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+        eps = rng.standard_normal((N, E)).astype(np.float32)
+        if bf16:
+            x, Wu, Wd = f32_to_bf16_bits(x), f32_to_bf16_bits(Wu), f32_to_bf16_bits(Wd)
+            x64, Wu64, Wd64 = (bf16_bits_to_f32(a).astype(np.float64) for a in (x, Wu, Wd))
+        else:
+            x64, Wu64, Wd64 = (a.astype(np.float64) for a in (x, Wu, Wd))
+        s_raw = oracle.router_logits(x, Wg, bg)
+        topk, _, s = oracle.route_from_logits(s_raw, k, eps if sigma else None, sigma, return_scores=True)
+        slot, _ = oracle.assign_slots(topk, E, oracle.capacity(N, E, k, cf))
+        assert (slot < 0).any() or cf >= 1.0
+        dy = rng.standard_normal((N, d))
+        got = oracle.backward(x, Wg, Wu, Wd, s, topk, slot, dy)
+        ref = _autograd_grads(x64, Wg.astype(np.float64), bg.astype(np.float64), Wu64, Wd64,
+                              eps.astype(np.float64), sigma, s, topk, slot, dy)
+        for name in ref:
+            scale = max(1.0, float(np.max(np.abs(ref[name]))))
+            assert np.max(np.abs(got[name] - ref[name])) <= 1e-12 * scale, (name, N, d, E, k)
+        if k == 1:
+            assert np.all(got["dW_g"] == 0.0) and np.all(got["db_g"] == 0.0)
+
+
 ALL_CHECKS = [check_m1, check_m2_slots, check_m2_combine, check_topk_bruteforce,
               check_gates_invariants, check_noise, check_capacity, check_slots_bruteforce,
               check_logits_vs_numpy, check_ffn_vs_numpy, check_dense_mixture,
               check_single_expert_mlp, check_all_dropped_is_zero, check_gelu_expert_variant,
-              check_gelu_bias_layer, check_load_stats_m2, check_load_stats_random]
+              check_gelu_bias_layer, check_load_stats_m2, check_load_stats_random, check_backward_vs_autograd]

@@ -22,8 +22,8 @@ MUTANTS = {
     "ties_to_higher_index": ("return (ia < ib) ? -1 : (ia > ib);", "return (ia > ib) ? -1 : (ia < ib);"),
     "ascending_scores": ("if (sa > sb) return -1;\n    if (sa < sb) return 1;",
                          "if (sa < sb) return -1;\n    if (sa > sb) return 1;"),
-    "softmax_over_all_experts": ("for (int j = 0; j < k; ++j)\n            denom +=",
-                                 "for (int j = 0; j < E; ++j)\n            denom +="),
+    "softmax_over_all_experts": ("for (int j = 0; j < k; ++j)\n            denom += exp((double)s[idx[j]]",
+                                 "for (int j = 0; j < E; ++j)\n            denom += exp((double)s[idx[j]]"),
     "relu_missing": ("h[f] = z > 0.0 ? z : 0.0;", "h[f] = z;"),
     "w_up_transposed": ("z += elem(W_up, dt, wrow + i)",
                         "z += elem(W_up, dt, (size_t)e * d_ff * d + (size_t)i * d_ff + f)"),
@@ -46,6 +46,15 @@ MUTANTS = {
                                  "denom += exp(top - (double)s[idx[j]]);"),
     "used_not_capped": ("used[e] = (int32_t)(q[e] < C ? q[e] : C);", "used[e] = (int32_t)q[e];"),
     "load_counts_once_per_token": ("            q[e] += 1;\n", "            q[e] += (j == 0);\n"),
+    "bwd_relu_mask_missing": ("                dz[f] = z[f] > 0.0 ? acc : 0.0;", "                dz[f] = acc;"),
+    "bwd_softmax_not_coupled": ("            const double ds = g[j] * (dg[j] - sum);",
+                                "            const double ds = g[j] * dg[j];"),
+    "bwd_dropped_choices_skipped": ("            const int e = ti[j];\n            db_g[e] += ds;",
+                                    "            const int e = ti[j];\n            if (slot[(size_t)t * k + j] < 0)\n"
+                                    "                continue;\n            db_g[e] += ds;"),
+    "bwd_router_to_x_missing": ("                dxt[i] += ds * (double)W_g[(size_t)e * d + i];", ""),
+    "bwd_dW_up_transposed": ("dW_up[((size_t)e * d_ff + f) * d + i] += dz[f] * elem(x, dt, (size_t)t * d + i);",
+                             "dW_up[((size_t)e * d + i) * d_ff + f] += dz[f] * elem(x, dt, (size_t)t * d + i);"),
     "gate_mass_truncated": ("mass[e] += llrint(ldexp((double)gates[(size_t)t * k + j], 32));",
                             "mass[e] += (int64_t)ldexp((double)gates[(size_t)t * k + j], 32);"),
 }
@@ -72,7 +81,7 @@ def test_pins_catch_mutant(tmp_path, name):
         mutant = ctypes.CDLL(lib_path)
         for fn in ("oracle_router_logits", "oracle_route_from_logits", "oracle_capacity",
                    "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine",
-                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex", "oracle_load_stats"):
+                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex", "oracle_load_stats", "oracle_backward"):
             getattr(mutant, fn).argtypes = getattr(saved, fn).argtypes
             getattr(mutant, fn).restype = getattr(saved, fn).restype
         O._lib = mutant
