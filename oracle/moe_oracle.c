@@ -171,11 +171,15 @@ void oracle_assign_slots(const int32_t *topk_idx, int64_t N, int E, int k, int64
  *     db_g[e] += ds_j,  dW_g[e] += ds_j x_t,  dx_t += ds_j W_g[e]
  * s [N, E] fp32 are the noisy scores the gates came from (s = s_raw + sigma eps:
  * ds_raw = ds); the gates are recomputed from them in double.  dy [N, d] double.
+ * relu_mask (nullable, [N, k, d_ff] bytes): the ReLU decisions [z > 0] of the
+ * kept pairs taken from elsewhere (another implementation's rounding of z),
+ * replayed in place of the sign of this oracle's own z: h = mask ? z : 0 and
+ * dz = mask ? W_down^T d_o : 0.  With NULL the oracle decides.
  * Outputs are double and overwritten: dx [N, d], dW_g [E, d], db_g [E],
  * dW_up [E, d_ff, d], dW_down [E, d, d_ff]. */
 void oracle_backward(const void *x, int dt, const float *W_g, const void *W_up, const void *W_down,
                      const float *s, const int32_t *topk_idx, const int32_t *slot, const double *dy,
-                     int64_t N, int d, int E, int d_ff, int k,
+                     int64_t N, int d, int E, int d_ff, int k, const uint8_t *relu_mask,
                      double *dx, double *dW_g, double *db_g, double *dW_up, double *dW_down)
 {
     memset(dx, 0, sizeof(double) * (size_t)N * d);
@@ -204,12 +208,14 @@ void oracle_backward(const void *x, int dt, const float *W_g, const void *W_up, 
             if (slot[(size_t)t * k + j] < 0)
                 continue;
             const int e = ti[j];
+            const uint8_t *mk = relu_mask ? relu_mask + ((size_t)t * k + j) * d_ff : NULL;
             for (int f = 0; f < d_ff; ++f) {
                 double acc = 0.0;
                 for (int i = 0; i < d; ++i)
                     acc += elem(W_up, dt, ((size_t)e * d_ff + f) * d + i) * elem(x, dt, (size_t)t * d + i);
                 z[f] = acc;
-                h[f] = acc > 0.0 ? acc : 0.0;
+                const int on = mk ? (mk[f] != 0) : (acc > 0.0);
+                h[f] = on ? acc : 0.0;
             }
             for (int i = 0; i < d; ++i) {
                 double acc = 0.0;
@@ -225,7 +231,7 @@ void oracle_backward(const void *x, int dt, const float *W_g, const void *W_up, 
                     dW_down[((size_t)e * d + i) * d_ff + f] += d_o * h[f];
                     acc += elem(W_down, dt, ((size_t)e * d + i) * d_ff + f) * d_o;
                 }
-                dz[f] = z[f] > 0.0 ? acc : 0.0;
+                dz[f] = (mk ? (mk[f] != 0) : (z[f] > 0.0)) ? acc : 0.0;
             }
             for (int f = 0; f < d_ff; ++f)
                 for (int i = 0; i < d; ++i) {
@@ -252,6 +258,235 @@ void oracle_backward(const void *x, int dt, const float *W_g, const void *W_up, 
     free(h);
     free(dz);
     free(o);
+}
+
+/* ------------------------------------------------------------------ sampled backward
+ * The quantities of oracle_backward at listed places only, for batches where
+ * the whole backward is too slow on a CPU: dx rows of listed tokens, rows f of
+ * dW_up[e] and columns f of dW_down[e] for listed (e, f), and all of dW_g and
+ * db_g.  Each listed value is summed in the same order as in oracle_backward
+ * (tokens ascending, then choices), so the two agree exactly.
+ *   tokens [n_tokens] -> dx_rows [n_tokens, d]
+ *   ef [n_ef, 2] (expert, f) -> dW_up_rows [n_ef, d] (= dW_up[e][f][:]) and
+ *                               dW_down_cols [n_ef, d] (= dW_down[e][:][f])
+ * The gate gradients of every kept pair (dg = dy . o) need every expert
+ * output, which is the expensive part: it runs on nthreads threads, split over
+ * tokens; the listed rows and columns are split over threads the same way. */
+struct bwd_ctx {
+    const void *x, *W_up, *W_down;
+    int dt;
+    const float *W_g, *s;
+    const int32_t *topk_idx, *slot;
+    const double *dy;
+    int64_t N;
+    int d, E, d_ff, k;
+    const uint8_t *relu_mask;
+    double *g, *dg, *ds;           /* [N, k] */
+    const int64_t *tokens;
+    const int32_t *ef;
+    double *dx_rows, *dW_up_rows, *dW_down_cols;
+};
+
+struct bwd_job {
+    struct bwd_ctx *c;
+    int64_t begin, end;
+};
+
+static int relu_on(const struct bwd_ctx *c, int64_t t, int j, int f, double z)
+{
+    if (c->relu_mask)
+        return c->relu_mask[((size_t)t * c->k + j) * c->d_ff + f] != 0;
+    return z > 0.0;
+}
+
+static double up_dot(const struct bwd_ctx *c, int e, int f, int64_t t)
+{
+    double acc = 0.0;
+    for (int i = 0; i < c->d; ++i)
+        acc += elem(c->W_up, c->dt, ((size_t)e * c->d_ff + f) * c->d + i) * elem(c->x, c->dt, (size_t)t * c->d + i);
+    return acc;
+}
+
+/* gates (recomputed in double from s) and dg = dy . o of every kept pair */
+static void *bwd_gate_grads(void *arg)
+{
+    struct bwd_job *jb = (struct bwd_job *)arg;
+    struct bwd_ctx *c = jb->c;
+    double *h = (double *)malloc(sizeof(double) * (size_t)c->d_ff);
+    for (int64_t t = jb->begin; t < jb->end; ++t) {
+        const int32_t *ti = c->topk_idx + (size_t)t * c->k;
+        const double top = (double)c->s[(size_t)t * c->E + ti[0]];
+        double denom = 0.0;
+        for (int j = 0; j < c->k; ++j)
+            denom += exp((double)c->s[(size_t)t * c->E + ti[j]] - top);
+        for (int j = 0; j < c->k; ++j)
+            c->g[(size_t)t * c->k + j] = exp((double)c->s[(size_t)t * c->E + ti[j]] - top) / denom;
+        const double *dyt = c->dy + (size_t)t * c->d;
+        for (int j = 0; j < c->k; ++j) {
+            double dgj = 0.0;
+            if (c->slot[(size_t)t * c->k + j] >= 0) {
+                const int e = ti[j];
+                for (int f = 0; f < c->d_ff; ++f) {
+                    const double z = up_dot(c, e, f, t);
+                    h[f] = relu_on(c, t, j, f, z) ? z : 0.0;
+                }
+                for (int i = 0; i < c->d; ++i) {
+                    double acc = 0.0;
+                    for (int f = 0; f < c->d_ff; ++f)
+                        acc += elem(c->W_down, c->dt, ((size_t)e * c->d + i) * c->d_ff + f) * h[f];
+                    dgj += dyt[i] * acc;
+                }
+            }
+            c->dg[(size_t)t * c->k + j] = dgj;
+        }
+    }
+    free(h);
+    return NULL;
+}
+
+/* dx rows of the listed tokens, in oracle_backward's order */
+static void *bwd_dx_rows(void *arg)
+{
+    struct bwd_job *jb = (struct bwd_job *)arg;
+    struct bwd_ctx *c = jb->c;
+    const int d = c->d, d_ff = c->d_ff, k = c->k;
+    double *z = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    double *dz = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    for (int64_t r = jb->begin; r < jb->end; ++r) {
+        const int64_t t = c->tokens[r];
+        const int32_t *ti = c->topk_idx + (size_t)t * k;
+        const double *dyt = c->dy + (size_t)t * d;
+        double *dxt = c->dx_rows + (size_t)r * d;
+        for (int i = 0; i < d; ++i)
+            dxt[i] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            if (c->slot[(size_t)t * k + j] < 0)
+                continue;
+            const int e = ti[j];
+            const double gj = c->g[(size_t)t * k + j];
+            for (int f = 0; f < d_ff; ++f)
+                z[f] = up_dot(c, e, f, t);
+            for (int f = 0; f < d_ff; ++f) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i)
+                    acc += elem(c->W_down, c->dt, ((size_t)e * d + i) * d_ff + f) * (gj * dyt[i]);
+                dz[f] = relu_on(c, t, j, f, z[f]) ? acc : 0.0;
+            }
+            for (int f = 0; f < d_ff; ++f)
+                for (int i = 0; i < d; ++i)
+                    dxt[i] += elem(c->W_up, c->dt, ((size_t)e * d_ff + f) * d + i) * dz[f];
+        }
+        for (int j = 0; j < k; ++j) {
+            const double dsj = c->ds[(size_t)t * k + j];
+            const int e = ti[j];
+            for (int i = 0; i < d; ++i)
+                dxt[i] += dsj * (double)c->W_g[(size_t)e * d + i];
+        }
+    }
+    free(z);
+    free(dz);
+    return NULL;
+}
+
+/* row f of dW_up[e] and column f of dW_down[e] for the listed (e, f) */
+static void *bwd_weight_rows(void *arg)
+{
+    struct bwd_job *jb = (struct bwd_job *)arg;
+    struct bwd_ctx *c = jb->c;
+    const int d = c->d, d_ff = c->d_ff, k = c->k;
+    for (int64_t q = jb->begin; q < jb->end; ++q) {
+        const int e = c->ef[2 * q], f = c->ef[2 * q + 1];
+        double *wu = c->dW_up_rows + (size_t)q * d;
+        double *wd = c->dW_down_cols + (size_t)q * d;
+        for (int i = 0; i < d; ++i)
+            wu[i] = wd[i] = 0.0;
+        for (int64_t t = 0; t < c->N; ++t) {
+            for (int j = 0; j < k; ++j) {
+                if (c->topk_idx[(size_t)t * k + j] != e || c->slot[(size_t)t * k + j] < 0)
+                    continue;
+                const double gj = c->g[(size_t)t * k + j];
+                const double *dyt = c->dy + (size_t)t * d;
+                const double z = up_dot(c, e, f, t);
+                const int on = relu_on(c, t, j, f, z);
+                const double hf = on ? z : 0.0;
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    const double d_o = gj * dyt[i];
+                    wd[i] += d_o * hf;
+                    acc += elem(c->W_down, c->dt, ((size_t)e * d + i) * d_ff + f) * d_o;
+                }
+                const double dzf = on ? acc : 0.0;
+                for (int i = 0; i < d; ++i)
+                    wu[i] += dzf * elem(c->x, c->dt, (size_t)t * d + i);
+            }
+        }
+    }
+    return NULL;
+}
+
+static void bwd_run(void *(*fn)(void *), struct bwd_ctx *c, int64_t n, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > n)
+        nthreads = n > 0 ? (int)n : 1;
+    struct bwd_job *jobs = (struct bwd_job *)calloc((size_t)nthreads, sizeof *jobs);
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof *th);
+    for (int w = 0; w < nthreads; ++w) {
+        jobs[w].c = c;
+        jobs[w].begin = n * w / nthreads;
+        jobs[w].end = n * (w + 1) / nthreads;
+    }
+    if (nthreads == 1) {
+        fn(&jobs[0]);
+    } else {
+        for (int w = 0; w < nthreads; ++w)
+            pthread_create(&th[w], NULL, fn, &jobs[w]);
+        for (int w = 0; w < nthreads; ++w)
+            pthread_join(th[w], NULL);
+    }
+    free(jobs);
+    free(th);
+}
+
+void oracle_backward_sampled(const void *x, int dt, const float *W_g, const void *W_up, const void *W_down,
+                             const float *s, const int32_t *topk_idx, const int32_t *slot, const double *dy,
+                             int64_t N, int d, int E, int d_ff, int k, const uint8_t *relu_mask,
+                             const int64_t *tokens, int64_t n_tokens, const int32_t *ef, int64_t n_ef,
+                             int nthreads, double *dx_rows, double *dW_g, double *db_g, double *dW_up_rows,
+                             double *dW_down_cols)
+{
+    struct bwd_ctx c;
+    memset(&c, 0, sizeof c);
+    c.x = x; c.W_up = W_up; c.W_down = W_down; c.dt = dt; c.W_g = W_g; c.s = s;
+    c.topk_idx = topk_idx; c.slot = slot; c.dy = dy; c.N = N; c.d = d; c.E = E; c.d_ff = d_ff; c.k = k;
+    c.relu_mask = relu_mask; c.tokens = tokens; c.ef = ef;
+    c.dx_rows = dx_rows; c.dW_up_rows = dW_up_rows; c.dW_down_cols = dW_down_cols;
+    c.g = (double *)malloc(sizeof(double) * (size_t)(N * k + 1));
+    c.dg = (double *)malloc(sizeof(double) * (size_t)(N * k + 1));
+    c.ds = (double *)malloc(sizeof(double) * (size_t)(N * k + 1));
+    bwd_run(bwd_gate_grads, &c, N, nthreads);
+    /* router gradients, in oracle_backward's order */
+    memset(dW_g, 0, sizeof(double) * (size_t)E * d);
+    memset(db_g, 0, sizeof(double) * (size_t)E);
+    for (int64_t t = 0; t < N; ++t) {
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j)
+            sum += c.g[(size_t)t * k + j] * c.dg[(size_t)t * k + j];
+        for (int j = 0; j < k; ++j) {
+            const double dsj = c.g[(size_t)t * k + j] * (c.dg[(size_t)t * k + j] - sum);
+            c.ds[(size_t)t * k + j] = dsj;
+            const int e = topk_idx[(size_t)t * k + j];
+            db_g[e] += dsj;
+            for (int i = 0; i < d; ++i)
+                dW_g[(size_t)e * d + i] += dsj * elem(x, dt, (size_t)t * d + i);
+        }
+    }
+    bwd_run(bwd_dx_rows, &c, n_tokens, nthreads);
+    bwd_run(bwd_weight_rows, &c, n_ef, nthreads);
+    free(c.g);
+    free(c.dg);
+    free(c.ds);
 }
 
 /* Per-expert load of one routed batch ("nanoMoEの深層解剖" slide 14: the

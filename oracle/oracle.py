@@ -52,8 +52,11 @@ def _load():
             lib.oracle_assign_slots.restype = None
             lib.oracle_load_stats.argtypes = [P, P, I64, I32, I32, I64, P, P, P]
             lib.oracle_load_stats.restype = None
-            lib.oracle_backward.argtypes = [P, I32, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, P, P, P, P, P]
+            lib.oracle_backward.argtypes = [P, I32, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, P, P, P, P, P, P]
             lib.oracle_backward.restype = None
+            lib.oracle_backward_sampled.argtypes = [P, I32, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, P,
+                                                    P, I64, P, I64, I32, P, P, P, P, P]
+            lib.oracle_backward_sampled.restype = None
             lib.oracle_expert_ffn.argtypes = [P, I32, P, P, I64, I32, I32, I32, P, P]
             lib.oracle_expert_ffn.restype = None
             lib.oracle_ffn_combine.argtypes = [P, I32, P, P, P, P, P, I32, I32, I32, P, I64, P, I32]
@@ -117,10 +120,19 @@ def assign_slots(topk_idx, E, C):
     return slot, counts
 
 
-def backward(x, W_g, W_up, W_down, s, topk_idx, slot, dy):
+def _mask(relu_mask, N, k, d_ff):
+    if relu_mask is None:
+        return None
+    m = np.ascontiguousarray(relu_mask, dtype=np.uint8)
+    assert m.shape == (N, k, d_ff)
+    return m
+
+
+def backward(x, W_g, W_up, W_down, s, topk_idx, slot, dy, relu_mask=None):
     """Gradients of L = sum(dy * y) for a given routing (STEP 6 and STEP 11):
     dict(dx [N,d], dW_g [E,d], db_g [E], dW_up [E,d_ff,d], dW_down [E,d,d_ff]), float64.
-    s [N,E] float32: the noisy scores the gates came from (route_from_logits' s_noisy)."""
+    s [N,E] float32: the noisy scores the gates came from (route_from_logits' s_noisy).
+    relu_mask [N,k,d_ff] (optional): ReLU decisions of the kept pairs to replay."""
     x = np.ascontiguousarray(x)
     W_g = np.ascontiguousarray(W_g, dtype=np.float32)
     W_up = np.ascontiguousarray(W_up)
@@ -134,9 +146,38 @@ def backward(x, W_g, W_up, W_down, s, topk_idx, slot, dy):
     k = topk_idx.shape[1]
     out = dict(dx=np.empty((N, d)), dW_g=np.empty((E, d)), db_g=np.empty(E), dW_up=np.empty((E, d_ff, d)),
                dW_down=np.empty((E, d, d_ff)))
+    mk = _mask(relu_mask, N, k, d_ff)
     _load().oracle_backward(_ptr(x), _dt(x), _ptr(W_g), _ptr(W_up), _ptr(W_down), _ptr(s), _ptr(topk_idx),
-                            _ptr(slot), _ptr(dy), N, d, E, d_ff, k, _ptr(out["dx"]), _ptr(out["dW_g"]),
+                            _ptr(slot), _ptr(dy), N, d, E, d_ff, k, _ptr(mk), _ptr(out["dx"]), _ptr(out["dW_g"]),
                             _ptr(out["db_g"]), _ptr(out["dW_up"]), _ptr(out["dW_down"]))
+    return out
+
+
+def backward_sampled(x, W_g, W_up, W_down, s, topk_idx, slot, dy, tokens, ef, relu_mask=None, nthreads=1):
+    """oracle_backward at listed places: dict(dx_rows [len(tokens), d],
+    dW_up_rows [len(ef), d] (dW_up[e, f, :]), dW_down_cols [len(ef), d]
+    (dW_down[e, :, f]), dW_g [E, d], db_g [E]), float64; ef: [(e, f), ...]."""
+    x = np.ascontiguousarray(x)
+    W_g = np.ascontiguousarray(W_g, dtype=np.float32)
+    W_up = np.ascontiguousarray(W_up)
+    W_down = np.ascontiguousarray(W_down)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    slot = np.ascontiguousarray(slot, dtype=np.int32)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    ef = np.ascontiguousarray(np.asarray(ef, dtype=np.int32).reshape(-1, 2))
+    N, d = x.shape
+    E, d_ff, _ = W_up.shape
+    k = topk_idx.shape[1]
+    mk = _mask(relu_mask, N, k, d_ff)
+    out = dict(dx_rows=np.empty((len(tokens), d)), dW_up_rows=np.empty((len(ef), d)),
+               dW_down_cols=np.empty((len(ef), d)), dW_g=np.empty((E, d)), db_g=np.empty(E))
+    _load().oracle_backward_sampled(_ptr(x), _dt(x), _ptr(W_g), _ptr(W_up), _ptr(W_down), _ptr(s),
+                                    _ptr(topk_idx), _ptr(slot), _ptr(dy), N, d, E, d_ff, k, _ptr(mk),
+                                    _ptr(tokens), len(tokens), _ptr(ef), len(ef), int(nthreads),
+                                    _ptr(out["dx_rows"]), _ptr(out["dW_g"]), _ptr(out["db_g"]),
+                                    _ptr(out["dW_up_rows"]), _ptr(out["dW_down_cols"]))
     return out
 
 

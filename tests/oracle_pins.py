@@ -473,8 +473,101 @@ def check_backward_vs_autograd(seed=15):
             assert np.all(got["dW_g"] == 0.0) and np.all(got["db_g"] == 0.0)
 
 
+def _small_routed_case(rng, N, d, E, d_ff, k, cf, sigma, bf16):
+    from sparse_mixture_experts_noisy_b200.synth import f32_to_bf16_bits
+    x = rng.standard_normal((N, d)).astype(np.float32)
+    Wg = rng.standard_normal((E, d)).astype(np.float32)
+    bg = rng.standard_normal(E).astype(np.float32)
+    Wu = rng.standard_normal((E, d_ff, d)).astype(np.float32)
+    Wd = rng.standard_normal((E, d, d_ff)).astype(np.float32)
+    eps = rng.standard_normal((N, E)).astype(np.float32)
+    if bf16:
+        x, Wu, Wd = f32_to_bf16_bits(x), f32_to_bf16_bits(Wu), f32_to_bf16_bits(Wd)
+    s_raw = oracle.router_logits(x, Wg, bg)
+    topk, _, s = oracle.route_from_logits(s_raw, k, eps if sigma else None, sigma, return_scores=True)
+    slot, _ = oracle.assign_slots(topk, E, oracle.capacity(N, E, k, cf))
+    dy = rng.standard_normal((N, d))
+    return x, Wg, Wu, Wd, s, topk, slot, dy
+
+
+def _z(x, Wu, topk, slot):
+    """z of every kept pair in float64 numpy: [N, k, d_ff] (0 for dropped)."""
+    from sparse_mixture_experts_noisy_b200.synth import bf16_bits_to_f32
+    f = (lambda a: bf16_bits_to_f32(a).astype(np.float64)) if x.dtype == np.uint16 else (lambda a: a.astype(np.float64))
+    x64, Wu64 = f(x), f(Wu)
+    N, k = topk.shape
+    z = np.zeros((N, k, Wu.shape[1]))
+    for t in range(N):
+        for j in range(k):
+            if slot[t, j] >= 0:
+                z[t, j] = Wu64[topk[t, j]] @ x64[t]
+    return z, x64
+
+
+def check_backward_sampled_matches_full(seed=21):
+    """The sampled backward gives exactly the full backward's numbers at the
+    listed tokens, dW_up rows and dW_down columns, and all of dW_g and db_g,
+    with the ReLU decisions taken by the oracle or replayed from a mask."""
+    rng = np.random.default_rng(seed)
+    for N, d, E, d_ff, k, cf, sigma, bf16 in ((11, 6, 4, 7, 2, 0.6, 0.5, True), (8, 5, 3, 4, 3, 0.7, 0.0, False)):
+        x, Wg, Wu, Wd, s, topk, slot, dy = _small_routed_case(rng, N, d, E, d_ff, k, cf, sigma, bf16)
+        z, _ = _z(x, Wu, topk, slot)
+        for mask in (None, (z > 0.1).astype(np.uint8)):
+            full = oracle.backward(x, Wg, Wu, Wd, s, topk, slot, dy, relu_mask=mask)
+            tokens = np.array([0, 3, N - 1])
+            ef = [(0, 0), (E - 1, d_ff - 1), (1, 2)]
+            got = oracle.backward_sampled(x, Wg, Wu, Wd, s, topk, slot, dy, tokens, ef, relu_mask=mask,
+                                          nthreads=3)
+            assert np.array_equal(got["dx_rows"], full["dx"][tokens])
+            assert np.array_equal(got["dW_g"], full["dW_g"]) and np.array_equal(got["db_g"], full["db_g"])
+            for q, (e, f) in enumerate(ef):
+                assert np.array_equal(got["dW_up_rows"][q], full["dW_up"][e, f, :])
+                assert np.array_equal(got["dW_down_cols"][q], full["dW_down"][e, :, f])
+
+
+def check_backward_relu_mask_replay(seed=23):
+    """A replayed ReLU mask equal to the oracle's own decisions changes
+    nothing; turning one decision off for a kept pair (t, j) at unit f takes
+    exactly dz_f x_t out of dW_up[e][f] and d_o z_f out of dW_down[e][:, f],
+    and changes dx only in row t (the decision acts on both h and dz)."""
+    rng = np.random.default_rng(seed)
+    N, d, E, d_ff, k = 9, 6, 3, 8, 2
+    x, Wg, Wu, Wd, s, topk, slot, dy = _small_routed_case(rng, N, d, E, d_ff, k, 1.0, 0.0, False)
+    z, x64 = _z(x, Wu, topk, slot)
+    own = (z > 0).astype(np.uint8)
+    base = oracle.backward(x, Wg, Wu, Wd, s, topk, slot, dy)
+    same = oracle.backward(x, Wg, Wu, Wd, s, topk, slot, dy, relu_mask=own)
+    for name in base:
+        assert np.array_equal(base[name], same[name]), name
+    t, j = 2, 0
+    assert slot[t, j] >= 0
+    f = int(np.argmax(z[t, j]))
+    assert z[t, j, f] > 0
+    off = own.copy()
+    off[t, j, f] = 0
+    got = oracle.backward(x, Wg, Wu, Wd, s, topk, slot, dy, relu_mask=off)
+    e = int(topk[t, j])
+    g = np.exp(s[t, topk[t]].astype(np.float64) - s[t, topk[t, 0]])
+    g = g / g.sum()
+    d_o = g[j] * dy[t]
+    Wd64 = Wd.astype(np.float64)
+    dz_f = float(Wd64[e][:, f] @ d_o)
+    du = base["dW_up"] - got["dW_up"]
+    dd = base["dW_down"] - got["dW_down"]
+    mask_up = np.zeros_like(du, dtype=bool)
+    mask_up[e, f, :] = True
+    mask_dn = np.zeros_like(dd, dtype=bool)
+    mask_dn[e, :, f] = True
+    assert np.all(du[~mask_up] == 0.0) and np.all(dd[~mask_dn] == 0.0)
+    np.testing.assert_allclose(du[e, f, :], dz_f * x64[t], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dd[e, :, f], d_o * z[t, j, f], rtol=1e-9, atol=1e-12)
+    ddx = base["dx"] - got["dx"]
+    assert np.all(ddx[np.arange(N) != t] == 0.0) and np.any(ddx[t] != 0.0)
+
+
 ALL_CHECKS = [check_m1, check_m2_slots, check_m2_combine, check_topk_bruteforce,
               check_gates_invariants, check_noise, check_capacity, check_slots_bruteforce,
               check_logits_vs_numpy, check_ffn_vs_numpy, check_dense_mixture,
               check_single_expert_mlp, check_all_dropped_is_zero, check_gelu_expert_variant,
-              check_gelu_bias_layer, check_load_stats_m2, check_load_stats_random, check_backward_vs_autograd]
+              check_gelu_bias_layer, check_load_stats_m2, check_load_stats_random, check_backward_vs_autograd,
+              check_backward_sampled_matches_full, check_backward_relu_mask_replay]

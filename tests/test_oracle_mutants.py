@@ -46,7 +46,14 @@ MUTANTS = {
                                  "denom += exp(top - (double)s[idx[j]]);"),
     "used_not_capped": ("used[e] = (int32_t)(q[e] < C ? q[e] : C);", "used[e] = (int32_t)q[e];"),
     "load_counts_once_per_token": ("            q[e] += 1;\n", "            q[e] += (j == 0);\n"),
-    "bwd_relu_mask_missing": ("                dz[f] = z[f] > 0.0 ? acc : 0.0;", "                dz[f] = acc;"),
+    "bwd_relu_mask_missing": ("                dz[f] = (mk ? (mk[f] != 0) : (z[f] > 0.0)) ? acc : 0.0;",
+                              "                dz[f] = acc;"),
+    "bwd_mask_not_replayed_in_h": ("const int on = mk ? (mk[f] != 0) : (acc > 0.0);", "const int on = (acc > 0.0);"),
+    "bwd_sampled_dx_relu_missing": ("dz[f] = relu_on(c, t, j, f, z[f]) ? acc : 0.0;", "dz[f] = acc;"),
+    "bwd_sampled_weight_rows_ungated": ("                    const double d_o = gj * dyt[i];\n                    wd[i]",
+                                        "                    const double d_o = dyt[i];\n                    wd[i]"),
+    "bwd_sampled_router_term_missing": ("                dxt[i] += dsj * (double)c->W_g[(size_t)e * d + i];",
+                                        "                dxt[i] += 0.0 * c->W_g[(size_t)e * d + i];"),
     "bwd_softmax_not_coupled": ("            const double ds = g[j] * (dg[j] - sum);",
                                 "            const double ds = g[j] * dg[j];"),
     "bwd_dropped_choices_skipped": ("            const int e = ti[j];\n            db_g[e] += ds;",
@@ -81,7 +88,8 @@ def test_pins_catch_mutant(tmp_path, name):
         mutant = ctypes.CDLL(lib_path)
         for fn in ("oracle_router_logits", "oracle_route_from_logits", "oracle_capacity",
                    "oracle_assign_slots", "oracle_expert_ffn", "oracle_ffn_combine",
-                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex", "oracle_load_stats", "oracle_backward"):
+                   "oracle_expert_ffn_ex", "oracle_ffn_combine_ex", "oracle_load_stats", "oracle_backward",
+                   "oracle_backward_sampled"):
             getattr(mutant, fn).argtypes = getattr(saved, fn).argtypes
             getattr(mutant, fn).restype = getattr(saved, fn).restype
         O._lib = mutant
