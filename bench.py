@@ -46,10 +46,15 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the secondary decode measurement")
+    ap.add_argument("--only", action="store_true", help="measure only --workload (no secondary workloads)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (small cases for profiling); implies --only")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if a.tokens is not None:
+        a.only = True
     return a
 
 
@@ -198,35 +203,6 @@ def ncu_traffic(kernel_tag: str):
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
-def oracle_sample_time(inp, wl, n_route: int, n_ffn: int, nthreads: int, rng):
-    """Times the oracle on a bounded sample and extrapolates to the whole batch.
-    Returns (seconds per batch, description)."""
-    import oracle
-    N = wl.N
-    n_route = max(1, min(n_route, N))
-    t0 = time.perf_counter()
-    lg = oracle.router_logits(inp.x[:n_route], inp.W_g, inp.b_g)
-    t_route = (time.perf_counter() - t0) * N / n_route
-    # routing + slot assignment on the full batch reuse the sampled logits
-    # pattern: tile the sample's logits to N rows (same arithmetic per row)
-    reps = int(math.ceil(N / n_route))
-    lg_full = np.tile(lg, (reps, 1))[:N]
-    noise = inp.noise
-    t0 = time.perf_counter()
-    idx, g = oracle.route_from_logits(lg_full, wl.k, noise, wl.sigma)
-    C = oracle.capacity(N, wl.E, wl.k, wl.cf)
-    slot, counts = oracle.assign_slots(idx, wl.E, C)
-    t_slots = time.perf_counter() - t0
-    toks = np.sort(rng.choice(N, size=max(1, min(n_ffn, N)), replace=False))
-    t0 = time.perf_counter()
-    oracle.ffn_combine(inp.x, inp.W_up, inp.W_down, idx, g, slot, tokens=toks, nthreads=nthreads)
-    t_ffn = (time.perf_counter() - t0) * N / len(toks)
-    desc = (f"router logits on {n_route} of {N} tokens, top-k/softmax/slots on all {N}, "
-            f"expert FFN + combine on {len(toks)} sampled tokens ({nthreads} threads); "
-            f"scaled to {N} tokens")
-    return t_route + t_slots + t_ffn, desc
-
-
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -234,10 +210,61 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def calibrated_ffn_tokens(wl, seconds: float, nthreads: int) -> int:
-    # about 1 ns per double multiply-add on one core for the oracle's plain loops
-    per_token = wl.k * 2.0 * wl.d * wl.d_ff * 1.0e-9
-    return max(1, min(wl.N, int(seconds * nthreads / max(per_token, 1e-9))))
+def oracle_tokens_for(wl, seconds: float, nthreads: int) -> int:
+    """Tokens of a sub-batch the oracle finishes in about `seconds`: the router
+    runs on one thread (d*E double multiply-adds per token), the expert FFN on
+    `nthreads` (k*2*d*d_ff per token), about 1 ns each."""
+    per_token = (wl.d * wl.E + wl.k * 2.0 * wl.d * wl.d_ff / max(1, nthreads)) * 1.0e-9
+    return max(1, min(wl.N, int(seconds / max(per_token, 1e-12))))
+
+
+class OracleSteps:
+    """The CPU oracle as the layer's reference implementation, on bounded
+    samples of the workload.  One step is the oracle's whole layer (router
+    logits, noise, KeepTopK, softmax, slot assignment against the sub-batch's
+    own capacity, expert FFN, combine) on a contiguous sub-batch of n tokens of
+    the workload's batch; successive steps take successive sub-batches.  Every
+    second of it is timed; nothing is extrapolated."""
+
+    def __init__(self, inp, wl, n, nthreads):
+        self.inp, self.wl, self.n, self.nthreads = inp, wl, n, nthreads
+        self.off = 0
+
+    def step(self) -> float:
+        import oracle
+        inp, wl = self.inp, self.wl
+        n = self.n
+        if self.off + n > wl.N:
+            self.off = 0
+        sl = slice(self.off, self.off + n)
+        noise = inp.noise[sl] if inp.noise is not None else None
+        t0 = time.perf_counter()
+        oracle.forward(inp.x[sl], inp.W_g, inp.b_g, noise, wl.sigma, wl.k, wl.cf, inp.W_up, inp.W_down,
+                       nthreads=self.nthreads)
+        dt = time.perf_counter() - t0
+        self.off += n
+        return dt
+
+    def describe(self) -> str:
+        wl = self.wl
+        whole = "the whole batch" if self.n == wl.N else f"contiguous {self.n}-token sub-batches of the {wl.N}-token batch"
+        return (f"oracle layer forward (logits, routing, slots with the sub-batch's own capacity, expert FFN, "
+                f"combine) on {whole}; FFN and combine on {self.nthreads} threads, the rest on one")
+
+
+def oracle_timed(inp, wl, seconds: float, nthreads: int, steps: int = 1, warmup: int = 1):
+    """Times `steps` oracle steps after `warmup` (the first warm-up step also
+    calibrates the sub-batch size to about `seconds` per step).
+    Returns (OracleSteps, total timed seconds, tokens timed)."""
+    n0 = oracle_tokens_for(wl, seconds, nthreads)
+    probe = OracleSteps(inp, wl, max(1, min(n0, max(1, n0 // 8))), nthreads)
+    t = probe.step()
+    n = max(1, min(wl.N, int(probe.n * seconds / max(t, 1e-6))))
+    run = OracleSteps(inp, wl, n, nthreads)
+    for _ in range(max(0, warmup - 1)):
+        run.step()
+    total = sum(run.step() for _ in range(steps))
+    return run, total, n * steps
 
 
 def run_reference(args):
@@ -248,27 +275,19 @@ def run_reference(args):
         return 0
     wl = WORKLOADS[args.workload]
     inp = make_inputs(wl, args.seed)
-    cores = cpu_cores()
-    nthreads = max(1, min(cores, 64))
-    rng = np.random.default_rng(args.seed)
-    n_ffn = calibrated_ffn_tokens(wl, 2.0, nthreads)
-    n_route = min(wl.N, 2048)
-    for _ in range(args.warmup):
-        oracle_sample_time(inp, wl, min(n_route, 64), 1, nthreads, rng)
-    times = []
-    desc = ""
-    for _ in range(args.steps):
-        t, desc = oracle_sample_time(inp, wl, n_route, n_ffn, nthreads, rng)
-        times.append(t)
-    sec = float(np.mean(times))
-    value = wl.N / sec
+    nthreads = max(1, min(cpu_cores(), 64))
+    # each step about 1.5 s of CPU work, so --steps 20 --warmup 5 ends within a minute or so
+    run, total, tokens = oracle_timed(inp, wl, 1.5, nthreads, steps=args.steps, warmup=args.warmup)
+    value = tokens / total
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                             "sample": desc},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                             "sample": run.describe(), "tokens_per_step": run.n},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            # not a measurement: the time a whole batch would take at the measured rate
+            "extrapolated_whole_batch_ms": 1e3 * total / tokens * wl.N}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -333,23 +352,27 @@ def measure_layer(wl, inp_dev, steps, warmup, dist, torch, moe, flush_needed):
     return graphed, y, sec, clk.summary()
 
 
-def measure_ffn(wl, inp_dev, steps, torch, moe):
+def measure_ffn(wl, inp_dev, steps, torch, moe, flush=None):
     """The dominant kernels alone: the expert FFN (tcgen05 grouped GEMMs) on the
-    batch's gathered rows, back to back on the current stream."""
+    batch's gathered rows, back to back on the current stream (the L2 flushed
+    between calls when `flush` is given)."""
     x, W_g, b_g, noise, W_up, W_down = inp_dev
     topk, gates, _ = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma, want_logits=False)
     dsp = moe.moe_dispatch(topk, x, wl.E, wl.cf)
     xg, offs, cnt = dsp["x_gathered"], dsp["offsets"], dsp["counts"]
     rows, d = xg.shape
     dt = moe.MOE_BF16 if xg.dtype == torch.bfloat16 else moe.MOE_F32
-    ws = torch.empty(moe.load_library().moe_expert_ffn_workspace_size(rows, d, wl.E, wl.d_ff, dt),
-                     dtype=torch.uint8, device=x.device)
+    ws = moe.new_workspace(moe.load_library().moe_expert_ffn_workspace_size(rows, d, wl.E, wl.d_ff, dt),
+                           x.device)
     out = torch.empty_like(xg)
     run = lambda: moe.moe_expert_ffn(xg, offs, cnt, W_up, W_down, ws=ws, out=out)  # noqa: E731
     for _ in range(3):
         run()
     torch.cuda.synchronize()
-    sec = time_steps(run, steps, torch)
+    sec = time_steps(run, steps, torch, flush)
+    code, word = moe.check_status(ws)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} (0x{word:08x}) after the expert FFN timing")
     counts = cnt.cpu().numpy().tolist()
     return sec / steps, counts
 
@@ -383,11 +406,74 @@ def measure_e2e(graphed, wl, inp, steps, torch, moe):
 
 
 def roofline_entry(kind, achieved, peak, unit, traffic, kernel, peak_src, extra=None):
-    e = {"bound": kind, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+    e = {"bound": kind, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": (achieved / peak) if peak else None,
          "traffic": traffic, "kernel": kernel, "peak_source": peak_src}
     if extra:
         e.update(extra)
     return e
+
+
+def ffn_kernel_name(wl, moe):
+    tc = wl.dtype == "bf16" and wl.d % 8 == 0 and wl.d_ff % 8 == 0
+    if not tc:
+        return "simt_gemm_kernel (fp32 CUDA cores, up + down)"
+    if moe.gathered_rows(wl.N, wl.E, wl.k, wl.cf) <= 256:
+        return "tc_gemm_kernel, weight-row tiles (up + down) + reduce_parts_kernel"
+    if os.environ.get("MOE_TC_PAIR", "1") != "0":
+        return "tc2_gemm_kernel, CTA pairs (up + down launches of one moe_expert_ffn call)"
+    return "tc_gemm_kernel (up + down launches of one moe_expert_ffn call)"
+
+
+def measure_workload(wl, inp_dev, steps, warmup, dist, dev, torch, moe, peaks, peak_src, ffn_steps):
+    """Device time of the graphed layer over `steps` steps (max over ranks),
+    the expert FFN alone for the roofline, and the clocks seen meanwhile."""
+    weights_bytes = 2 * wl.E * wl.d * wl.d_ff * (2 if wl.dtype == "bf16" else 4)
+    flush_needed = weights_bytes <= L2_BYTES
+    graphed, _, sec, clocks = measure_layer(wl, inp_dev, steps, warmup, dist, torch, moe, flush_needed)
+    max_sec = dist.max(sec, device=dev)
+    agg = aggregate(wl.N, steps, dist.world, max_sec)
+    step_s = max_sec / steps
+    elem = 2 if wl.dtype == "bf16" else 4
+    kernel = ffn_kernel_name(wl, moe)
+    flush = None
+    if flush_needed:
+        buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush = lambda: buf.fill_(1)  # noqa: E731
+    ffn_sec, counts = measure_ffn(wl, inp_dev, ffn_steps, torch, moe, flush)
+    R = int(sum(counts))
+    decode_plan = "weight-row" in kernel
+    if wl.dtype != "bf16":
+        # fp32 storage: CUDA-core FFMA; a handful of tokens is launch-latency bound
+        fl = ffn_flops(R, wl.d, wl.d_ff)
+        roof = roofline_entry("latency", step_s * 1e6, None, "us", None, kernel, None,
+                              {"ffn_us_per_call": ffn_sec * 1e6, "algorithmic_flops": fl, "kept_rows": R,
+                               "note": "fp32 toy layer: the step is a few kernel launches, no roofline applies"})
+    elif decode_plan:
+        byt = ffn_bytes(counts, wl.d, wl.d_ff, elem)
+        layer_bytes = byt + wl.N * wl.d * elem * 2 + wl.E * wl.d * 4
+        roof = roofline_entry("hbm", byt / ffn_sec / 1e9, peaks["hbm_gbs"], "GB/s", ncu_traffic("decode"),
+                              kernel, peak_src + " (copy)",
+                              {"algorithmic_bytes": byt, "ms_per_call": ffn_sec * 1e3,
+                               "whole_layer_gbs": layer_bytes / step_s / 1e9,
+                               "whole_layer_frac": layer_bytes / step_s / 1e9 / peaks["hbm_gbs"],
+                               "whole_layer_frac_of_8tbs": layer_bytes / step_s / 8e12})
+    else:
+        fl = ffn_flops(R, wl.d, wl.d_ff)
+        roof = roofline_entry("tensor", fl / ffn_sec / 1e12, peaks["bf16_tflops"], "TFLOP/s",
+                              ncu_traffic("prefill_" + wl.name), kernel, peak_src + " burst",
+                              {"frac_of_sustained": fl / ffn_sec / 1e12 / peaks["bf16_tflops_sustained"],
+                               "algorithmic_flops": fl, "kept_rows": R, "ms_per_call": ffn_sec * 1e3,
+                               "whole_layer_frac": fl / step_s / 1e12 / peaks["bf16_tflops"]})
+    out = {"workload": wl.name, "value": agg["value"], "unit": UNIT, "ms_per_step": agg["ms_per_step"],
+           "steps": steps, "config": workload_config(wl), "roofline": roof, "clocks": clocks,
+           "gpu_launches": moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) * steps}
+    return out, graphed
+
+
+# timed steps of the secondary workloads, whatever --steps is: enough that the
+# timed region lasts about half a second and the clock sampler sees 20 samples
+SECONDARY_STEPS = {"decode": 1500, "nano": 2500, "fine": 200, "toy": 5000}
 
 
 def run_ours(args):
@@ -400,101 +486,66 @@ def run_ours(args):
     dev = torch.device("cuda", dist.local_rank)
     moe.load_library()
     peaks, peak_src = load_peaks()
-    wl = WORKLOADS[args.workload]
-    # replicas of one model: the same weights on every rank, each rank its own tokens
-    inp = make_inputs(wl, args.seed)
-    if dist.rank > 0:
-        inp.x = make_x(wl, args.seed + 7919 * dist.rank)
-        inp.noise = make_noise(wl, args.seed + 7919 * dist.rank)
+
+    def inputs(name, weights=True):
+        wl = WORKLOADS[name]
+        if args.tokens is not None and name == args.workload:
+            wl = wl.with_(N=args.tokens)
+        # replicas of one model: the same weights on every rank, each rank its own tokens
+        inp = make_inputs(wl, args.seed, weights=weights)
+        if dist.rank > 0:
+            inp.x = make_x(wl, args.seed + 7919 * dist.rank)
+            inp.noise = make_noise(wl, args.seed + 7919 * dist.rank)
+        return wl, inp
+
+    wl, inp = inputs(args.workload)
     inp_dev = tuple(to_dev(a, torch) for a in (inp.x, inp.W_g, inp.b_g, inp.noise, inp.W_up, inp.W_down))
-    weights_bytes = 2 * wl.E * wl.d * wl.d_ff * (2 if wl.dtype == "bf16" else 4)
-    flush = weights_bytes <= L2_BYTES
-
-    layer, y, sec, clocks = measure_layer(wl, inp_dev, args.steps, args.warmup, dist, torch, moe, flush)
-    max_sec = dist.max(sec, device=dev)
-    agg = aggregate(wl.N, args.steps, dist.world, max_sec)
-
-    # the dominant kernels alone
-    ffn_steps = max(10, min(args.steps, 200))
-    ffn_sec, counts = measure_ffn(wl, inp_dev, ffn_steps, torch, moe)
-    R = int(sum(counts))
-    elem = 2 if wl.dtype == "bf16" else 4
-    tc = wl.dtype == "bf16" and wl.d % 8 == 0 and wl.d_ff % 8 == 0
-    decode_plan = tc and moe.gathered_rows(wl.N, wl.E, wl.k, wl.cf) <= 256
-    if not tc:
-        kernel = "simt_gemm_kernel (up + down)"
-    elif os.environ.get("MOE_TC_PAIR", "1") != "0":
-        kernel = "tc2_gemm_kernel, CTA pairs (up + down launches of one moe_expert_ffn call)"
-    else:
-        kernel = "tc_gemm_kernel (up + down launches of one moe_expert_ffn call)"
-    if decode_plan:
-        byt = ffn_bytes(counts, wl.d, wl.d_ff, elem)
-        roof = roofline_entry("hbm", byt / ffn_sec / 1e9, peaks["hbm_gbs"], "GB/s",
-                              ncu_traffic("decode"), "tc_gemm_kernel, weight-row tiles (up + down) + reduce_parts_kernel",
-                              peak_src + " (copy)",
-                              {"algorithmic_bytes": byt, "ms_per_call": ffn_sec * 1e3})
-    else:
-        fl = ffn_flops(R, wl.d, wl.d_ff)
-        roof = roofline_entry("tensor", fl / ffn_sec / 1e12, peaks["bf16_tflops"], "TFLOP/s",
-                              ncu_traffic("prefill_" + wl.name), kernel, peak_src + " burst",
-                              {"frac_of_sustained": fl / ffn_sec / 1e12 / peaks["bf16_tflops_sustained"],
-                               "algorithmic_flops": fl, "kept_rows": R, "ms_per_call": ffn_sec * 1e3})
-        layer_tflops = fl / (max_sec / args.steps) / 1e12
-        roof["whole_layer_frac"] = layer_tflops / peaks["bf16_tflops"]
+    main, graphed = measure_workload(wl, inp_dev, args.steps, args.warmup, dist, dev, torch, moe, peaks, peak_src,
+                                     max(10, min(args.steps, 200)))
 
     # end to end through the public API with host buffers
     e2e_steps = max(5, min(args.steps, 50))
-    e2e_sec, h2d, d2h = measure_e2e(layer, wl, inp, e2e_steps, torch, moe)
+    e2e_sec, h2d, d2h = measure_e2e(graphed, wl, inp, e2e_steps, torch, moe)
     e2e_sec = dist.max(e2e_sec, device=dev)
 
-    line = {"metric": METRIC, "value": agg["value"], "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
+    line = {"metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": workload_config(wl, {"parallelism": f"replicas x{dist.world}" if dist.world > 1 else "1 GPU",
                                            "seed": args.seed}),
-            "roofline": roof,
+            "roofline": main["roofline"],
             "e2e": {"value": wl.N * dist.world / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) * args.steps,
-            "clocks": clocks}
+            "gpu_launches": main["gpu_launches"],
+            "clocks": main["clocks"]}
+    del graphed
 
-    # the decode-shaped workload shares the weights' shapes and seeds with the
-    # Mixtral-shaped one; measure it too when running that workload
-    if args.workload == "mixtral" and not args.no_decode:
-        dwl = WORKLOADS["decode"]
-        dinp = make_inputs(dwl, args.seed + 7919 * dist.rank, weights=False)
-        ddev = (to_dev(dinp.x, torch), inp_dev[1], None, None, inp_dev[4], inp_dev[5])
-        dsteps = max(20, args.steps)
-        dlayer, _, dsec, dclk = measure_layer(dwl, ddev, dsteps, args.warmup, dist, torch, moe, False)
-        dmax = dist.max(dsec, device=dev)
-        dagg = aggregate(dwl.N, dsteps, dist.world, dmax)
-        fsec, dcounts = measure_ffn(dwl, ddev, dsteps, torch, moe)
-        byt = ffn_bytes(dcounts, dwl.d, dwl.d_ff, 2)
-        layer_bytes = byt + dwl.N * dwl.d * 2 * 2 + dwl.E * dwl.d * 4
-        line["decode"] = {
-            "workload": "decode", "value": dagg["value"], "unit": UNIT, "ms_per_step": dagg["ms_per_step"],
-            "steps": dsteps,
-            "roofline": roofline_entry("hbm", byt / fsec / 1e9, peaks["hbm_gbs"], "GB/s", ncu_traffic("decode"),
-                                       "tc_gemm_kernel (decode tiles, up + down) + reduce_parts_kernel",
-                                       peak_src + " (copy)",
-                                       {"algorithmic_bytes": byt, "ms_per_call": fsec * 1e3,
-                                        "whole_layer_gbs": layer_bytes / (dmax / dsteps) / 1e9,
-                                        "whole_layer_frac": layer_bytes / (dmax / dsteps) / 1e9 / peaks["hbm_gbs"],
-                                        "whole_layer_frac_of_8tbs": layer_bytes / (dmax / dsteps) / 8e12}),
-            "clocks": dclk,
-            # the decode run's own timed region (the top-level count is the main one's)
-            "gpu_launches": moe.forward_launches(dwl.N, dwl.d, dwl.E, dwl.d_ff, dwl.k, dwl.cf,
-                                                 ddev[0].dtype) * dsteps}
+    # every other workload, each with its own timed region, roofline and clocks
+    if args.workload == "mixtral" and not args.only:
+        for name in ("decode", "nano", "fine", "toy"):
+            if name == "decode" and args.no_decode:
+                continue
+            if name == "decode":
+                # same weight shapes and seeds as the Mixtral-shaped layer: reuse them
+                swl, sinp = inputs("decode", weights=False)
+                sdev = (to_dev(sinp.x, torch), inp_dev[1], None, None, inp_dev[4], inp_dev[5])
+            else:
+                swl, sinp = inputs(name)
+                sdev = tuple(to_dev(a, torch) for a in (sinp.x, sinp.W_g, sinp.b_g, sinp.noise, sinp.W_up,
+                                                        sinp.W_down))
+            steps = SECONDARY_STEPS[name]
+            obj, g = measure_workload(swl, sdev, steps, args.warmup, dist, dev, torch, moe, peaks, peak_src,
+                                      max(20, min(steps, 200)))
+            del g, sdev
+            obj.pop("config")
+            line[name] = obj
+            torch.cuda.empty_cache()
 
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        cores = cpu_cores()
-        nthreads = max(1, min(cores, 64))
-        rng = np.random.default_rng(args.seed)
-        n_ffn = calibrated_ffn_tokens(wl, args.cpu_seconds * 0.7, nthreads)
-        n_route = min(wl.N, max(256, int(args.cpu_seconds * 0.2 * 1e9 / max(1, wl.E * wl.d))))
-        t, desc = oracle_sample_time(inp, wl, n_route, n_ffn, nthreads, rng)
-        line["cpu_baseline"] = {"value": wl.N / t, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                                "sample": desc}
+        nthreads = max(1, min(cpu_cores(), 64))
+        run, total, tokens = oracle_timed(inp, wl, args.cpu_seconds, nthreads, steps=1, warmup=1)
+        line["cpu_baseline"] = {"value": tokens / total, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                                "sample": run.describe() + f" ({run.n} tokens, {total:.1f} s timed)"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

@@ -31,8 +31,14 @@
  *    moe_last_error() (thread-local, valid until the next call on that
  *    thread).  Argument errors are detected on the host before anything is
  *    launched.  Kernel-side failures (a bounded wait that ran out, an index
- *    check) are recorded in the workspace's status word and returned by
- *    moe_check_status().  No kernel traps.
+ *    check) are recorded in a status word and returned by moe_check_status()
+ *    (or moe_check_route_status() for moe_route).  No kernel traps.
+ *  - The status word is the first 4 bytes of a workspace (or the word given to
+ *    moe_route_ex).  Kernels only OR error bits into it; nothing but
+ *    moe_check_status() clears it, so an error stays visible through any
+ *    number of later calls until the caller reads it.  A fresh workspace's
+ *    first 4 bytes must be zeroed once before its first use (cudaMemset, or a
+ *    moe_check_status() call, which reads and then clears the word).
  *  - Preconditions: 1 <= k <= E <= 256; N >= 0; d, d_ff >= 1; inputs finite
  *    (NaN or Inf in the scores gives unspecified routing).
  *  - Ties in the top-k go to the lower expert index; the k kept experts of a
@@ -100,10 +106,33 @@ MOE_API int64_t moe_gathered_rows(int64_t N, int E, int k, double cf);
  * exactly into three bf16 parts, so every product is exact and only the fp32
  * accumulation rounds; other shapes run on CUDA cores.  Either way the top-k
  * and softmax are the same given the logits, and a token's results do not
- * depend on N or on its position in the batch. */
+ * depend on N or on its position in the batch.
+ *
+ * Every wait in the tensor-core router is bounded (1 s).  If one runs out, the
+ * kernel writes expert -1 and gate 0 for the tokens it could not finish and
+ * records MOE_ERR_TIMEOUT: moe_route in the library's own per-device status
+ * word, read and cleared by moe_check_route_status(); moe_route_ex in the
+ * caller's word.  Concurrent moe_route calls share the library's word, so a
+ * caller that needs per-call attribution uses moe_route_ex. */
 MOE_API moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                      const float *noise, float sigma, int64_t N, int d, int E, int k,
                      float *logits_out, int32_t *topk_idx, float *gates, void *stream);
+
+/* moe_route with the caller's status word: `status` (device, 16-byte aligned,
+ * at least 4 bytes, zero before first use; NULL selects the library's word as
+ * in moe_route) receives the error bits, and moe_check_status(status, ...)
+ * reads and clears it.  A workspace of moe_forward can serve: its status word
+ * is its first 4 bytes. */
+MOE_API moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                                const float *noise, float sigma, int64_t N, int d, int E, int k,
+                                float *logits_out, int32_t *topk_idx, float *gates, void *status,
+                                void *stream);
+
+/* Synchronises `stream` after reading and clearing (on that stream) the
+ * library's status word of moe_route calls on the current device.  Returns
+ * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *detail (nullable) receives
+ * the raw word. */
+MOE_API moe_status moe_check_route_status(void *stream, uint32_t *detail);
 
 /* ---------------------------------------------------------------- dispatch */
 
@@ -144,8 +173,11 @@ MOE_API moe_status moe_dispatch(const int32_t *topk_idx, const void *x, moe_dtyp
  * 8 MiB, i.e. about N * k * E > 2^29) get MOE_ERR_INVALID_ARG with a
  * message.  The call allocates nothing and calls no allocating routine.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) for that device; make that first call before any
- *    stream capture on the device.
+ *    (cudaGetSymbolAddress) for that device, which loads the library's device
+ *    code there if it is not loaded yet; make that first call before any
+ *    stream capture on the device.  The address is kept per device and CUDA
+ *    context: after cudaDeviceReset (a new context) the next call looks it up
+ *    again, so make a first call again before capturing.
  *  - Every call shares the one array and leaves its contents behind; the
  *    passes overwrite every scratch entry they read, so nothing has to start
  *    at zero.
@@ -230,6 +262,17 @@ MOE_API moe_status moe_expert_ffn_ex(const void *x_gathered, const int32_t *offs
                                      int d_ff, int E, int activation, const float *b_up, const float *b_down,
                                      void *out_gathered, void *ws, size_t ws_bytes, void *stream);
 
+/* The expert FFN of a training step: as moe_expert_ffn (ReLU, no biases), and
+ * the hidden activations H [rows, d_ff] of dt (device, caller-owned) are kept
+ * for moe_backward: H[r] = ReLU(W_up[e] x_gathered[r]) rounded to dt, rows
+ * outside the kept ranges unspecified.  out_gathered is written in every plan
+ * (the decode plan sums its K-split partials into it).  Same workspace as
+ * moe_expert_ffn. */
+MOE_API moe_status moe_expert_ffn_train(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                                        const void *W_up, const void *W_down, moe_dtype dt, int64_t rows, int d,
+                                        int d_ff, int E, void *out_gathered, void *H, void *ws, size_t ws_bytes,
+                                        void *stream);
+
 /* ---------------------------------------------------------------- combine */
 
 /* Gate-weighted combine back to token order ("Mixture of Experts (MoE) 12段階…"
@@ -262,6 +305,52 @@ MOE_API size_t moe_load_stats_workspace_size(void);
 MOE_API moe_status moe_load_stats(const int32_t *topk_idx, const float *gates, int64_t N, int E, int k,
                                   double cf, int32_t *load, int32_t *used, double *importance, void *ws,
                                   size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- backward */
+
+/* Workspace bytes for moe_backward. */
+MOE_API size_t moe_backward_workspace_size(int64_t N, int d, int E, int d_ff, int k, int64_t rows, moe_dtype dt);
+
+/* Gradients of L = sum over t, i of dy[t][i] y[t][i] for the routing of a
+ * forward pass made with the staged calls (moe_route, moe_dispatch,
+ * moe_expert_ffn_train, moe_combine), ReLU experts without biases.
+ * ("Mixture of Experts (MoE) 12段階…" STEP 6: the -inf mask keeps the kept
+ * experts' softmax differentiable; STEP 11: g_i E_i(x) carries the gradient
+ * to the router; "nanoMoEの深層解剖" slide 10: the router is trained by
+ * backpropagation.)  The top-k indices and slots carry no gradient.  For a
+ * kept pair (t, j) of expert e and gathered row r:
+ *   dg = dy_t . O_r,  dO_r = g_j dy_t,  dZ_r = (dO_r W_down[e]) * [H_r > 0],
+ *   dX_r = dZ_r W_up[e],  dW_down[e] += dO_r^T H_r,  dW_up[e] += dZ_r^T x_gathered_r;
+ * for every chosen pair (dropped ones too, with dg = 0, since the gates are
+ * formed before the capacity cut): ds_j = g_j (dg_j - sum_l g_l dg_l),
+ *   dW_g[e] += ds_j x_t,  db_g[e] += ds_j,  dx_t = sum_kept dX_r + sum_j ds_j W_g[e_j].
+ * The noise is added to the scores, so these are also the gradients through
+ * the pre-noise logits.
+ *
+ *  x, W_g, W_up, W_down, N, d, E, d_ff, k   the forward's inputs
+ *  rows                     moe_gathered_rows() of the forward
+ *  topk_idx, gates          device [N, k] from moe_route
+ *  slot, offsets, counts    device, from moe_dispatch
+ *  x_gathered               device [rows, d] of dt, from moe_dispatch
+ *  H                        device [rows, d_ff] of dt, from moe_expert_ffn_train
+ *  out_gathered             device [rows, d] of dt, from moe_expert_ffn_train
+ *  dy                       device [N, d] of dt
+ *  dx                       device [N, d] of dt out
+ *  dW_g [E, d], db_g [E], dW_up [E, d_ff, d], dW_down [E, d, d_ff]   device fp32 out
+ *                           (overwritten; an expert without rows gets zeros)
+ *  ws, ws_bytes             workspace of moe_backward_workspace_size() bytes; its first
+ *                           4 bytes are the status word (moe_check_status)
+ * bf16 with d and d_ff multiples of 8: the four expert GEMMs run on the tensor
+ * cores (fp32 accumulation; dO, dZ and the expert part of dx rounded to bf16
+ * on the way, weight gradients in fp32); otherwise fp32 CUDA-core kernels.
+ * Deterministic: no atomics decide a sum's order. */
+MOE_API moe_status moe_backward(const void *x, moe_dtype dt, const float *W_g, const void *W_up,
+                                const void *W_down, int64_t N, int d, int E, int d_ff, int k, int64_t rows,
+                                const int32_t *topk_idx, const float *gates, const int32_t *slot,
+                                const int32_t *offsets, const int32_t *counts, const void *x_gathered,
+                                const void *H, const void *out_gathered, const void *dy, void *dx, float *dW_g,
+                                float *db_g, float *dW_up, float *dW_down, void *ws, size_t ws_bytes,
+                                void *stream);
 
 /* ---------------------------------------------------------------- fused */
 
@@ -298,19 +387,22 @@ MOE_API int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, doubl
 
 /* ---------------------------------------------------------------- status */
 
-/* Synchronises `stream` and reads the status word at the start of a workspace
- * given to moe_expert_ffn or moe_forward.  Returns MOE_OK, MOE_ERR_TIMEOUT (a
- * bounded wait in a kernel ran out; the kernel skipped its remaining work and
- * released its tensor memory) or MOE_ERR_DEVICE_CHECK.  *detail (nullable)
- * receives the raw word.  Clears the word. */
+/* Reads the status word at the start of a workspace given to moe_expert_ffn,
+ * moe_forward or moe_debug_wait_timeout (or a word given to moe_route_ex),
+ * clears it, both on `stream`, and synchronises the stream.  Returns MOE_OK,
+ * MOE_ERR_TIMEOUT (a bounded wait in a kernel ran out since the word was last
+ * cleared; that kernel skipped its remaining work and released its tensor
+ * memory) or MOE_ERR_DEVICE_CHECK.  *detail (nullable) receives the raw word:
+ * bit 0 timeout, bit 2 index check, bits 8-15 which wait ran out (ORed). */
 MOE_API moe_status moe_check_status(void *ws, void *stream, uint32_t *detail);
 
 /* Diagnostic for the bounded-wait machinery: launches one CTA that waits on
  * a shared-memory barrier nothing will ever complete, with a limit of
  * timeout_us microseconds, using the same wait routine as the tensor-core
- * kernels.  The kernel then records MOE_ERR_TIMEOUT in the status word of ws
- * (>= 256 bytes) and returns.  No pages' counterpart; exists so that tests
- * can check that a wait which runs out ends cleanly. */
+ * kernels.  The kernel then ORs MOE_ERR_TIMEOUT's bit into the status word of
+ * ws (>= 256 bytes) and returns.  No pages' counterpart; exists so that tests
+ * can check that a wait which runs out ends cleanly and that its report
+ * survives later calls on the same workspace. */
 MOE_API moe_status moe_debug_wait_timeout(uint32_t timeout_us, void *ws, size_t ws_bytes, void *stream);
 
 /* Number of streaming multiprocessors the library sizes its persistent grids

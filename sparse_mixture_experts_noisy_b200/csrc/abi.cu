@@ -6,6 +6,8 @@
 #include <mutex>
 #include <string>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "internal.h"
@@ -106,10 +108,13 @@ FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows,
     return L;
 }
 
+// H_keep (nullable): the caller's [rows][d_ff] buffer for the hidden
+// activations; null keeps them in the workspace.
 moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts, const void *W_up,
                    const void *W_down, moe_dtype dt, int64_t rows, int d, int d_ff, int E, void *out,
                    void *ffn_ws, bool combine_reads_parts, float **parts_out, int *nparts_out,
-                   uint32_t *status, cudaStream_t s, int act, const float *b_up, const float *b_down) {
+                   uint32_t *status, cudaStream_t s, int act, const float *b_up, const float *b_down,
+                   void *H_keep = nullptr) {
     cudaError_t e;
     if (parts_out) *parts_out = nullptr;
     if (nparts_out) *nparts_out = 0;
@@ -117,7 +122,7 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
         const int sms = num_sms_current();
         const moe::TcPlan p = moe::plan_tc_ffn(rows, d, d_ff, E, sms);
         uint8_t *w = static_cast<uint8_t *>(ffn_ws);
-        void *H = w;
+        void *H = H_keep ? H_keep : w;
         float *parts = p.decode ? reinterpret_cast<float *>(w + moe::align_up(static_cast<size_t>(rows) * d_ff * 2, 256))
                                 : nullptr;
         e = moe::launch_tc_ffn(xg, offsets, counts, W_up, W_down, rows, d, d_ff, E, out, H, parts,
@@ -130,7 +135,7 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
         return MOE_OK;
     }
     e = moe::launch_simt_ffn(xg, offsets, counts, W_up, W_down, dt == MOE_BF16 ? 1 : 0, rows, d, d_ff,
-                             E, out, ffn_ws, s, act, b_up, b_down);
+                             E, out, H_keep ? H_keep : ffn_ws, s, act, b_up, b_down);
     if (e != cudaSuccess) return cuda_fail(e, "CUDA-core expert FFN launch");
     return MOE_OK;
 }
@@ -142,22 +147,55 @@ moe_status run_ffn(const void *xg, const int32_t *offsets, const int32_t *counts
 constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress, once per device, with that device current.
+// Unique id of the calling thread's current CUDA context (0 if there is none
+// yet).  Context ids are never reused within a process, unlike the handles.
+unsigned long long current_context_id() {
+    static const auto fns = [] {
+        struct F {
+            PFN_cuCtxGetCurrent_v4000 get = nullptr;
+            PFN_cuCtxGetId_v12000 id = nullptr;
+        } f;
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.get = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            f.id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+        return f;
+    }();
+    if (fns.get == nullptr || fns.id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    if (fns.get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    unsigned long long id = 0;
+    if (fns.id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_noalloc_scratch in the current device's context.  In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with cudaGetSymbolAddress, with the device current, once per
+// device and context: a new context (after cudaDeviceReset, say) reloads the
+// module, which may place the array elsewhere, so its address is looked up
+// again.
 cudaError_t noalloc_scratch_address(void **out) {
     static std::mutex mu;
     static void *addr[64] = {nullptr};
+    static unsigned long long ctx_of[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+    const unsigned long long ctx = current_context_id();
+    if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // creates the context if needed
         if (e != cudaSuccess) return e;
         addr[dev] = p;
+        ctx_of[dev] = current_context_id();
     }
     *out = addr[dev];
     return cudaSuccess;
@@ -185,9 +223,9 @@ int64_t moe_gathered_rows(int64_t N, int E, int k, double cf) {
     return rows_for(N, E, k, C);
 }
 
-moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
-                     const float *noise, float sigma, int64_t N, int d, int E, int k,
-                     float *logits_out, int32_t *topk_idx, float *gates, void *stream) {
+moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                        const float *noise, float sigma, int64_t N, int d, int E, int k,
+                        float *logits_out, int32_t *topk_idx, float *gates, void *status, void *stream) {
     moe_status st = check_shape(N, d, E, k, dt);
     if (st != MOE_OK) return st;
     if (N > 0) {
@@ -199,11 +237,30 @@ moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float 
         OPTIONAL_PTR(noise, "noise");
         OPTIONAL_PTR(logits_out, "logits_out");
     }
+    OPTIONAL_PTR(status, "status");
     if (!std::isfinite(sigma)) return fail(MOE_ERR_INVALID_ARG, "sigma must be finite");
     cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
-                                      logits_out, topk_idx, gates, nullptr,
+                                      logits_out, topk_idx, gates, static_cast<uint32_t *>(status),
                                       static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
+    return MOE_OK;
+}
+
+moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
+                     const float *noise, float sigma, int64_t N, int d, int E, int k,
+                     float *logits_out, int32_t *topk_idx, float *gates, void *stream) {
+    return moe_route_ex(x, dt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, nullptr, stream);
+}
+
+moe_status moe_check_route_status(void *stream, uint32_t *detail) {
+    uint32_t word = 0;
+    cudaError_t e = moe::route_status_read_clear(&word, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "router status read");
+    if (detail) *detail = word;
+    if (word & moe::ST_TIMEOUT)
+        return fail(MOE_ERR_TIMEOUT, "a router wait ran out (status 0x%08x)", word);
+    if (word & moe::ST_BOUNDS)
+        return fail(MOE_ERR_DEVICE_CHECK, "a router index check failed (status 0x%08x)", word);
     return MOE_OK;
 }
 
@@ -363,12 +420,93 @@ moe_status moe_expert_ffn_ex(const void *x_gathered, const int32_t *offsets, con
     REQUIRE_PTR(ws, "ws");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t *status = static_cast<uint32_t *>(ws);
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), s);
-    if (e != cudaSuccess) return cuda_fail(e, "status reset");
     if (rows == 0) return MOE_OK;
     return run_ffn(x_gathered, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, out_gathered,
                    static_cast<uint8_t *>(ws) + moe::kStatusBytes, false, nullptr, nullptr, status, s, activation,
                    b_up, b_down);
+}
+
+moe_status moe_expert_ffn_train(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
+                                const void *W_up, const void *W_down, moe_dtype dt, int64_t rows, int d,
+                                int d_ff, int E, void *out_gathered, void *H, void *ws, size_t ws_bytes,
+                                void *stream) {
+    if (dt != MOE_F32 && dt != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 or MOE_BF16");
+    if (rows < 0 || rows % 128 != 0)
+        return fail(MOE_ERR_INVALID_ARG, "rows must be a non-negative multiple of 128 (moe_gathered_rows)");
+    if (d < 1 || d_ff < 1 || E < 1 || E > 256) return fail(MOE_ERR_INVALID_ARG, "bad d, d_ff or E");
+    if (rows > INT32_MAX) return fail(MOE_ERR_INVALID_ARG, "rows must fit in int32");
+    REQUIRE_PTR(offsets, "offsets");
+    REQUIRE_PTR(counts, "counts");
+    REQUIRE_PTR(W_up, "W_up");
+    REQUIRE_PTR(W_down, "W_down");
+    if (rows > 0) {
+        REQUIRE_PTR(x_gathered, "x_gathered");
+        REQUIRE_PTR(out_gathered, "out_gathered");
+        REQUIRE_PTR(H, "H");
+    }
+    const size_t need = moe::kStatusBytes + ffn_ws_bytes(rows, d, E, d_ff, dt);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "expert FFN workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    if (rows == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return run_ffn(x_gathered, offsets, counts, W_up, W_down, dt, rows, d, d_ff, E, out_gathered,
+                   static_cast<uint8_t *>(ws) + moe::kStatusBytes, false, nullptr, nullptr,
+                   static_cast<uint32_t *>(ws), s, MOE_ACT_RELU, nullptr, nullptr, H);
+}
+
+size_t moe_backward_workspace_size(int64_t N, int d, int E, int d_ff, int k, int64_t rows, moe_dtype dt) {
+    if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1 || rows < 0) return 0;
+    moe::BwdArgs a{};
+    a.dt = dt == MOE_BF16 ? 1 : 0;
+    a.N = N; a.d = d; a.E = E; a.d_ff = d_ff; a.k = k; a.rows = rows;
+    return moe::bwd_layout(a, num_sms_current()).total;
+}
+
+moe_status moe_backward(const void *x, moe_dtype dt, const float *W_g, const void *W_up, const void *W_down,
+                        int64_t N, int d, int E, int d_ff, int k, int64_t rows, const int32_t *topk_idx,
+                        const float *gates, const int32_t *slot, const int32_t *offsets, const int32_t *counts,
+                        const void *x_gathered, const void *H, const void *out_gathered, const void *dy,
+                        void *dx, float *dW_g, float *db_g, float *dW_up, float *dW_down, void *ws,
+                        size_t ws_bytes, void *stream) {
+    moe_status st = check_shape(N, d, E, k, dt);
+    if (st != MOE_OK) return st;
+    if (d_ff < 1) return fail(MOE_ERR_INVALID_ARG, "d_ff must be >= 1");
+    if (rows < 0 || rows % 128 != 0 || rows > INT32_MAX)
+        return fail(MOE_ERR_INVALID_ARG, "rows must be a non-negative multiple of 128 that fits in int32");
+    REQUIRE_PTR(W_g, "W_g");
+    REQUIRE_PTR(W_up, "W_up");
+    REQUIRE_PTR(W_down, "W_down");
+    REQUIRE_PTR(dW_g, "dW_g");
+    REQUIRE_PTR(db_g, "db_g");
+    REQUIRE_PTR(dW_up, "dW_up");
+    REQUIRE_PTR(dW_down, "dW_down");
+    REQUIRE_PTR(offsets, "offsets");
+    REQUIRE_PTR(counts, "counts");
+    if (N > 0) {
+        REQUIRE_PTR(x, "x");
+        REQUIRE_PTR(topk_idx, "topk_idx");
+        REQUIRE_PTR(gates, "gates");
+        REQUIRE_PTR(slot, "slot");
+        REQUIRE_PTR(dy, "dy");
+        REQUIRE_PTR(dx, "dx");
+        REQUIRE_PTR(x_gathered, "x_gathered");
+        REQUIRE_PTR(H, "H");
+        REQUIRE_PTR(out_gathered, "out_gathered");
+    }
+    moe::BwdArgs a{x, dt == MOE_BF16 ? 1 : 0, W_g, W_up, W_down, N, d, E, d_ff, k, rows, topk_idx, gates, slot,
+                   offsets, counts, x_gathered, H, out_gathered, dy, dx, dW_g, db_g, dW_up, dW_down};
+    const int sms = num_sms_current();
+    const size_t need = moe::bwd_layout(a, sms).total;
+    if (ws == nullptr || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "backward workspace needs %zu bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    REQUIRE_PTR(ws, "ws");
+    cudaError_t e = moe::launch_backward(a, ws, static_cast<uint32_t *>(ws), kWaitTimeoutNs, sms,
+                                         use_tensor_cores(dt, d, d_ff), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return MOE_OK;
 }
 
 moe_status moe_expert_ffn(const void *x_gathered, const int32_t *offsets, const int32_t *counts,
@@ -532,13 +670,13 @@ int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, mo
 moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {
     if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "ws must not be NULL");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     uint32_t word = 0;
-    e = cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost);
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "status read");
-    e = cudaMemset(ws, 0, sizeof word);
+    e = cudaMemsetAsync(ws, 0, sizeof word, s);
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     if (detail) *detail = word;
     if (word & moe::ST_TIMEOUT)
         return fail(MOE_ERR_TIMEOUT, "a kernel's bounded wait ran out (status 0x%08x)", word);
@@ -553,9 +691,8 @@ moe_status moe_debug_wait_timeout(uint32_t timeout_us, void *ws, size_t ws_bytes
     if (timeout_us == 0 || timeout_us > 2000000u)
         return fail(MOE_ERR_INVALID_ARG, "timeout_us must be in [1, 2000000]");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
-    if (e == cudaSuccess)
-        e = moe::launch_wait_timeout(static_cast<uint32_t *>(ws), static_cast<uint64_t>(timeout_us) * 1000ull, s);
+    cudaError_t e =
+        moe::launch_wait_timeout(static_cast<uint32_t *>(ws), static_cast<uint64_t>(timeout_us) * 1000ull, s);
     if (e != cudaSuccess) return cuda_fail(e, "wait-timeout diagnostic launch");
     return MOE_OK;
 }

@@ -11,11 +11,17 @@
 namespace moe {
 
 // ---------------------------------------------------------------- status word
-// The first 4 bytes of a workspace.  Kernels OR bits into it; the host reads it
-// with moe_check_status().
+// The first 4 bytes of a workspace.  Kernels only OR error bits into it and
+// never clear it; moe_check_status() reads and clears it, so an error stays
+// visible across later calls until the host looks.
+//
+// Inside a kernel the waits work on a per-CTA copy in shared memory: a role
+// that gives up sets ST_ABORT there so the CTA's other roles stop early, and
+// at exit one thread ORs the error bits (never ST_ABORT) into the global word.
+// An abort therefore never leaks into another CTA or a later launch.
 enum : uint32_t {
     ST_TIMEOUT = 1u << 0,      // a bounded wait ran out
-    ST_ABORT = 1u << 1,        // another role gave up; stop early
+    ST_ABORT = 1u << 1,        // another role of this CTA gave up; stop early (CTA-local only)
     ST_BOUNDS = 1u << 2,       // an index check failed
     ST_WHERE_SHIFT = 8,        // bits 8..15: which wait ran out (diagnostic)
 };
@@ -81,9 +87,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete, for at most
-// timeout_ns of wall-clock time.  Returns false if the wait ran out (the
-// status word then carries ST_TIMEOUT | ST_ABORT and `where`) or if another
-// role of the kernel already gave up (ST_ABORT seen).  Never spins forever.
+// timeout_ns of wall-clock time.  `status` is the CTA's shared-memory status
+// copy.  Returns false if the wait ran out (the copy then carries
+// ST_TIMEOUT | ST_ABORT and `where`) or if another role of the CTA already
+// gave up (ST_ABORT seen).  Never spins forever.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   uint32_t *status, uint64_t timeout_ns,
                                                   uint32_t where) {
@@ -113,6 +120,13 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, ui
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok;
+}
+
+// ORs a CTA's error bits (without ST_ABORT) into the global status word.
+// Call from one thread after the CTA's roles are done.
+__device__ __forceinline__ void publish_status(uint32_t *global, uint32_t cta_word) {
+    const uint32_t v = cta_word & ~static_cast<uint32_t>(ST_ABORT);
+    if (v != 0u && global != nullptr) atomicOr(global, v);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -146,6 +160,16 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void *tmap,
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 
@@ -218,6 +242,25 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by TMA
+// with 128-byte swizzling: each 128-byte row holds 64 consecutive M (or N)
+// elements of one K index, and 8 such rows make a 1024-byte swizzle atom.
+// lbo: bytes between successive 64-element blocks along M (or N); sbo: bytes
+// between successive groups of 8 K rows.  Other fields as for K-major.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
+// Instruction-descriptor bits that mark A (bit 15) or B (bit 16) as MN-major.
+constexpr uint32_t kIdescAMajorMN = 1u << 15;
+constexpr uint32_t kIdescBMajorMN = 1u << 16;
+
 // Instruction descriptor for kind::f16 with bf16 A and B (both K-major), fp32 D:
 // D format F32 (bits 4-5 = 1), A format BF16 (7-9 = 1), B format BF16 (10-12 = 1),
 // N >> 3 (17-22), M >> 4 (24-28).
@@ -253,19 +296,21 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
 }
 // TMA tile load into this CTA's shared memory whose completion bytes go to the
 // pair leader's mbarrier `bar` (a cluster-window address).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *tmap, uint32_t bar, int x, int y) {
+// `policy`: an L2 eviction policy from createpolicy (policy_evict_*).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *tmap, uint32_t bar, int x, int y,
+                                                 uint64_t policy) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "l"(0x1000000000000000ull)
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap, uint32_t bar, int x, int y,
-                                                 int z) {
+                                                 int z, uint64_t policy) {
     asm volatile(
         "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(0x1000000000000000ull)
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {

@@ -47,8 +47,9 @@ constexpr int kThreads = 192;
 
 // Epilogues: bf16 out with the optional bias (down projection), bf16 out with
 // bias and activation (up projection), raw fp32 partial sums (K splits; bias
-// and activation are applied once the splits are added).
-enum { EPI_BF16 = 0, EPI_BF16_ACT = 1, EPI_F32 = 2 };
+// and activation are applied once the splits are added), bf16 out zeroed
+// where a mask array is not positive (the ReLU's derivative in the backward).
+enum { EPI_BF16 = 0, EPI_BF16_ACT = 1, EPI_F32 = 2, EPI_BF16_MASK = 3 };
 
 struct TcArgs {
     const int32_t *offsets;
@@ -61,6 +62,10 @@ struct TcArgs {
     uint64_t timeout_ns;
     const float *bias;  // [E][Nw] fp32 or null: added to every output row of expert e
     int act;            // EPI_BF16_ACT: 1 = ReLU, 2 = GELU (x * Phi(x))
+    int group_m;        // pair tiles: M tiles per raster group (0 = all of the expert's)
+    int l2_hint;        // pair tiles: 0 both operands evict_normal; 1 token rows evict_last;
+                        // 2 token rows evict_last, weights evict_first
+    const __nv_bfloat16 *mask;  // EPI_BF16_MASK: [rows][Nw], same layout as out
 };
 
 __device__ __forceinline__ float activate(float v, int act) {
@@ -161,11 +166,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
     __shared__ uint32_t tmem_holder;
     __shared__ int32_t pre_s[257];
     __shared__ int32_t cnt_s[256];
+    __shared__ uint32_t cta_status;  // this CTA's copy of the status word
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E, Nw = args.Nw, splits = args.splits;
     const int kb_total = (args.K + kBK - 1) / kBK;
-    uint32_t *status = args.status;
+    uint32_t *status = &cta_status;
     const uint64_t tmo = args.timeout_ns;
 
     const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -187,6 +193,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
         mbar_init(tempty0 + 8, 4);
         mbar_init(drain, 1);
         fence_barrier_init();
+        cta_status = 0u;
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_tok);
@@ -396,6 +403,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
     }
     __syncwarp();
     __syncthreads();
+    if (threadIdx.x == 0) publish_status(args.status, cta_status);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
@@ -413,7 +421,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant
 // drain their own accumulators and report to the leader's barrier.  Per byte
 // moved from L2 this does a third more MMA work than the one-CTA tile, and each
 // stage is 32 KB, so the ring is 50 % deeper.
-template <int EPI, int STAGES>
+//
+// B_MN: the weights are stored [E][K][Nw] (K rows, Nw contiguous), as the
+// backward reads W_down and W_up; each CTA then loads its 128 weight columns
+// as two 64-wide MN-major boxes and the MMA reads B MN-major.
+template <int EPI, int STAGES, bool B_MN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
                 const TcArgs args) {
@@ -428,6 +440,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     __shared__ uint32_t tmem_holder;
     __shared__ int32_t pre_s[257];
     __shared__ int32_t cnt_s[256];
+    __shared__ uint32_t cta_status;  // this CTA's copy of the status word
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -435,7 +448,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int E = args.E, Nw = args.Nw, splits = args.splits;
     const int kb_total = (args.K + kBK - 1) / kBK;
-    uint32_t *status = args.status;
+    uint32_t *status = &cta_status;
     const uint64_t tmo = args.timeout_ns;
 
     const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -459,6 +472,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
         mbar_init(tempty0 + 8, 8);
         mbar_init(drain, 1);
         fence_barrier_init();
+        cta_status = 0u;
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_tok);
@@ -496,9 +510,21 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
         int r = u - pre_s[lo];
         const int split = r % splits;
         r /= splits;
+        // Raster: the expert's M tiles in groups of at most group_m (balanced);
+        // inside a group M tiles fastest, then N tiles.  Units in flight at
+        // one time then share a few token-row tiles and a few weight tiles.
         const int mt = (cnt_s[lo] + BT - 1) / BT;
-        tok0 = (r % mt) * BT;
-        w0 = (r / mt) * BT;
+        const int nt = (Nw + BT - 1) / BT;
+        const int G = (args.group_m > 0 && args.group_m < mt) ? args.group_m : mt;
+        const int ng = (mt + G - 1) / G;
+        const int q = r / nt;  // group i holds units [m0(i) * nt, m0(i + 1) * nt)
+        int gi = static_cast<int>(static_cast<int64_t>(q) * ng / mt);
+        while (gi > 0 && gi * mt / ng > q) --gi;
+        while ((gi + 1) * mt / ng <= q) ++gi;
+        const int m0 = gi * mt / ng, gs = (gi + 1) * mt / ng - m0;
+        const int rr = r - m0 * nt;
+        tok0 = (m0 + rr % gs) * BT;
+        w0 = (rr / gs) * BT;
         n_valid = min(BT, Nw - w0);
         kb0 = static_cast<int>(static_cast<int64_t>(split) * kb_total / splits);
         kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * kb_total / splits);
@@ -511,6 +537,8 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
             uint32_t phase = 0;
             bool ok = true;
             int issued = 0;
+            const uint64_t pol_tok = args.l2_hint >= 1 ? policy_evict_last() : policy_evict_normal();
+            const uint64_t pol_w = args.l2_hint >= 2 ? policy_evict_first() : policy_evict_normal();
             for (int u = pair; u < total_units && ok; u += npairs) {
                 int e, tok0, w0, kb0, kb1, nv;
                 decode(u, e, tok0, w0, kb0, kb1, nv);
@@ -525,8 +553,13 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
                     const uint32_t fb = full0_lead + 8 * stage;
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
                     const int kx = kb * kBK;
-                    tma_load_2d_pair(sa, &tm_tok, fb, kx, tok_row);
-                    tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, kx, w_row, e);
+                    tma_load_2d_pair(sa, &tm_tok, fb, kx, tok_row, pol_tok);
+                    if constexpr (B_MN) {
+                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, w_row, kx, e, pol_w);
+                        tma_load_3d_pair(sa + A_BYTES + 8192u, &tm_w, fb, w_row + 64, kx, e, pol_w);
+                    } else {
+                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, kx, w_row, e, pol_w);
+                    }
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -556,7 +589,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
             uint32_t phase = 0;
             bool ok = true, any = false;
             int local = 0;
-            const uint32_t idesc = idesc_bf16_f32(256, 256);
+            const uint32_t idesc = idesc_bf16_f32(256, 256) | (B_MN ? kIdescBMajorMN : 0u);
             for (int u = pair; u < total_units && ok; u += npairs) {
                 int e, tok0, w0, kb0, kb1, nv;
                 decode(u, e, tok0, w0, kb0, kb1, nv);
@@ -576,10 +609,14 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
                     tc_fence_after();
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
                     const uint64_t ad = smem_desc_sw128(sa);
-                    const uint64_t bd = smem_desc_sw128(sa + A_BYTES);
+                    // MN-major B: 64-wide N blocks 8 KB apart, 8-row K groups 1 KB
+                    // apart; the next 16 K rows start 2 KB on (+128 in the field)
+                    const uint64_t bd = B_MN ? smem_desc_mn_sw128(sa + A_BYTES, 8192u, 1024u)
+                                             : smem_desc_sw128(sa + A_BYTES);
+                    constexpr uint32_t bstep = B_MN ? 128u : 2u;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_pair(d_tmem, ad + 2 * kk, bd + bstep * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
                     any = true;
                     umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
                     if (++stage == STAGES) {
@@ -621,6 +658,21 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
                 tmem_wait_ld();
                 bias_act<EPI, false>(r, args, e, w0 + c * 32, 0);
                 const int col0 = w0 + c * 32;
+                if constexpr (EPI == EPI_BF16_MASK) {
+                    if (rv) {
+                        const __nv_bfloat16 *mk = args.mask + grow * args.ldo + col0;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (col0 + 8 * g < Nw) {
+                                uint4 mv = *reinterpret_cast<const uint4 *>(mk + 8 * g);
+                                const __nv_bfloat16 *mb = reinterpret_cast<const __nv_bfloat16 *>(&mv);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    if (!(__bfloat162float(mb[i]) > 0.0f)) r[8 * g + i] = 0u;
+                            }
+                        }
+                    }
+                }
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(args.out) + grow * args.ldo;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -647,6 +699,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
     }
     __syncwarp();
     __syncthreads();
+    if (threadIdx.x == 0) publish_status(args.status, cta_status);
     cluster_sync();  // the pair's MMAs and remote arrivals are done before TMEM goes
     if (warp == 1) {
         tc_fence_after();
@@ -670,20 +723,47 @@ cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, i
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act};
+    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act, 0, 0,
+             nullptr};
     return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, tm_tok, tm_w, a);
 }
 
-template <int EPI, int STAGES>
+// Raster group and L2 policies of the pair tiles for a GEMM of depth K.
+// MOE_TC_GROUP_M and MOE_TC_L2HINT override them (for measurements).
+struct TcRaster {
+    int group_m, l2_hint;
+};
+TcRaster tc2_raster(int K) {
+    static const int env_group = [] {
+        const char *v = getenv("MOE_TC_GROUP_M");
+        return v ? atoi(v) : -1;
+    }();
+    static const int env_hint = [] {
+        const char *v = getenv("MOE_TC_L2HINT");
+        return v ? atoi(v) : -1;
+    }();
+    (void)K;
+    TcRaster r{0, 0};
+    if (env_group >= 0) r.group_m = env_group;
+    if (env_hint >= 0) r.l2_hint = env_hint;
+    return r;
+}
+
+template <int EPI, int STAGES, bool B_MN = false>
 cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, int Nw, int K,
                        const int32_t *offsets, const int32_t *counts, void *out, int64_t ldo,
                        uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s,
-                       const float *bias = nullptr, int act = 1) {
+                       const float *bias = nullptr, int act = 1, const void *mask = nullptr) {
     CUtensorMap tm_tok, tm_w;
     if (!make_tmap_bf16_2d(&tm_tok, tok, tok_rows, K, 128)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
+    if (B_MN) {
+        // W is [E][K][Nw]: boxes of 64 weight columns x 64 K rows
+        if (!make_tmap_bf16_3d(&tm_w, W, E, K, Nw, 64)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_tmap_bf16_3d(&tm_w, W, E, Nw, K, 128)) return cudaErrorInvalidValue;
+    }
     constexpr int smem = STAGES * 2 * 128 * kBK * 2 + 1024;
-    auto kern = tc2_gemm_kernel<EPI, STAGES>;
+    auto kern = tc2_gemm_kernel<EPI, STAGES, B_MN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int pairs = num_sms / 2;
@@ -697,8 +777,288 @@ cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, 
         max_clusters < pairs)
         pairs = max_clusters;
     (void)cudaGetLastError();
-    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns, bias, act};
+    const TcRaster rs = tc2_raster(K);
+    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns, bias, act, rs.group_m, rs.l2_hint,
+             static_cast<const __nv_bfloat16 *>(mask)};
     return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), smem, s, tm_tok, tm_w, a);
+}
+
+// ---------------------------------------------------------------- weight gradients
+// D[e][m][n] = sum over expert e's gathered rows r of P[r][m] * Q[r][n], fp32
+// out: the backward's dW_down[e] = dO^T H and dW_up[e] = dZ^T X.  The GEMM's
+// K is the expert's rows, so both operands are read MN-major: per 64-row K
+// block the CTA loads its 128 columns of P (two 64-wide boxes, A) and 256
+// columns of Q (four boxes, B).  The rows of a K block past the expert's last
+// row belong to the next expert (the layout has no padding): before the MMAs
+// of that block the MMA warp overwrites those K rows with zeros in shared
+// memory.  An expert without rows gets a zero tile without MMAs.
+// Warp roles as in tc_gemm_kernel; units (expert, M tile, N tile), with the
+// operand whose tile set is smaller walked fastest so it stays in L2.
+struct WgArgs {
+    const int32_t *offsets;
+    const int32_t *counts;
+    int E, M, Nn;  // D[e] is [M][Nn]
+    int m_fast;    // 1: M tiles fastest
+    float *out;
+    uint32_t *status;
+    uint64_t timeout_ns;
+};
+
+constexpr int kWM = 128, kWN = 256;
+
+template <int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_wgrad_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
+                const WgArgs args) {
+    constexpr uint32_t A_BYTES = kWM * kBK * 2;   // two 8 KB boxes
+    constexpr uint32_t B_BYTES = kWN * kBK * 2;   // four 8 KB boxes
+    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t TMEM_COLS = 2 * kWN;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+    __shared__ uint32_t tmem_holder;
+    __shared__ int32_t cnt_s[256];
+    __shared__ int32_t off_s[256];
+    __shared__ uint32_t cta_status;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E, M = args.M, Nn = args.Nn;
+    const int mt = (M + kWM - 1) / kWM, nt = (Nn + kWN - 1) / kWN;
+    const int total_units = E * mt * nt;
+    uint32_t *status = &cta_status;
+    const uint64_t tmo = args.timeout_ns;
+
+    const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
+    const uint32_t full0 = smem_u32(&bars[0]);
+    const uint32_t empty0 = smem_u32(&bars[STAGES]);
+    const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
+    const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(tfull0, 1);
+        mbar_init(tfull0 + 8, 1);
+        mbar_init(tempty0, 4);
+        mbar_init(tempty0 + 8, 4);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+        cta_status = 0u;
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_p);
+        tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        cnt_s[e] = args.counts[e];
+        off_s[e] = args.offsets[e];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_holder;
+
+    auto decode = [&](int u, int &e, int &m, int &n) {
+        e = u / (mt * nt);
+        const int r = u - e * (mt * nt);
+        if (args.m_fast) {
+            m = r % mt;
+            n = r / mt;
+        } else {
+            m = r / nt;
+            n = r % nt;
+        }
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+                int e, m, n;
+                decode(u, e, m, n);
+                const int nk = (cnt_s[e] + kBK - 1) / kBK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 31)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full0 + 8 * stage;
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    const int y = off_s[e] + kb * kBK;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) tma_load_2d(sa + h * 8192u, &tm_p, fb, m * kWM + h * 64, y);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        tma_load_2d(sa + A_BYTES + h * 8192u, &tm_q, fb, n * kWN + h * 64, y);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && i < issued; ++i) {
+                    if (st == 0) {
+                        st = STAGES - 1;
+                        ph ^= 1u;
+                    } else {
+                        --st;
+                    }
+                    wait_drain(full0 + 8 * st, ph, tmo);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ tail zeroing + MMA issue (whole warp)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, any = false;
+        int local = 0;
+        const uint32_t idesc = idesc_bf16_f32(kWM, kWN) | kIdescAMajorMN | kIdescBMajorMN;
+        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            int e, m, n;
+            decode(u, e, m, n);
+            const int cnt = cnt_s[e];
+            const int nk = (cnt + kBK - 1) / kBK;
+            if (nk == 0) continue;
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            if (!mbar_wait_warp(tempty0 + 8 * acc, acc_phase ^ 1u, status, tmo, 32)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kWN);
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!mbar_wait_warp(full0 + 8 * stage, phase, status, tmo, 33)) {
+                    ok = false;
+                    break;
+                }
+                const int v = cnt - kb * kBK;  // valid K rows of this block
+                if (v < kBK) {
+                    uint8_t *st = smem_gen + stage * STAGE_BYTES;
+                    const int per_box = (kBK - v) * 8;  // 16-byte chunks past the last row
+                    for (int q = lane; q < 6 * per_box; q += 32) {
+                        const int box = q / per_box, rem = q - box * per_box;
+                        *reinterpret_cast<uint4 *>(st + box * 8192 + (v + rem / 8) * 128 + (rem % 8) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();  // the zeros, visible to the MMA
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint64_t ad = smem_desc_mn_sw128(sa, 8192u, 1024u);
+                    const uint64_t bd = smem_desc_mn_sw128(sa + A_BYTES, 8192u, 1024u);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16(d_tmem, ad + 128u * kk, bd + 128u * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(empty0 + 8 * stage);
+                }
+                any = true;
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(tfull0 + 8 * acc);
+            ++local;
+        }
+        if (!ok && any && lane == 0) {
+            umma_commit(drain);
+            wait_drain(drain, 0, tmo);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+            int e, m, n;
+            decode(u, e, m, n);
+            const int mrow = m * kWM + row_in_tile;
+            float *o = args.out + (static_cast<int64_t>(e) * M + mrow) * Nn;
+            if (cnt_s[e] == 0) {
+                // no rows: a zero gradient, without touching the tensor memory
+                if (mrow < M)
+                    for (int c = n * kWN; c < n * kWN + kWN && c < Nn; c += 4)
+                        *reinterpret_cast<float4 *>(o + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+                continue;
+            }
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            if (!mbar_wait_warp(tfull0 + 8 * acc, acc_phase, status, tmo, 34)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(acc * kWN);
+            for (int c = 0; c < kWN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_wait_ld();
+                const int col0 = n * kWN + c * 32;
+                if (mrow < M) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int col = col0 + 4 * g;
+                        if (col < Nn)
+                            *reinterpret_cast<float4 *>(o + col) =
+                                make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                            __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+            ++local;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (threadIdx.x == 0) publish_status(args.status, cta_status);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+cudaError_t launch_wgrad(const void *P, const void *Q, int64_t rows, int M, int Nn, const int32_t *offsets,
+                         const int32_t *counts, int E, float *out, uint32_t *status, uint64_t timeout_ns,
+                         int num_sms, cudaStream_t s) {
+    constexpr int STAGES = 4;
+    CUtensorMap tm_p, tm_q;
+    if (!make_tmap_bf16_2d(&tm_p, P, rows, M, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tm_q, Q, rows, Nn, 64)) return cudaErrorInvalidValue;
+    constexpr int smem = STAGES * (kWM + kWN) * kBK * 2 + 1024;
+    auto kern = tc_wgrad_kernel<STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int units = E * ((M + kWM - 1) / kWM) * ((Nn + kWN - 1) / kWN);
+    const int grid = units < num_sms ? units : num_sms;
+    WgArgs a{offsets, counts, E, M, Nn, M <= Nn ? 1 : 0, out, status, timeout_ns};
+    return launch_pdl(kern, dim3(grid > 0 ? grid : 1), dim3(kThreads), smem, s, tm_p, tm_q, a);
 }
 
 // Sum of K-split fp32 partials into bf16 rows, in split order, then the
@@ -840,17 +1200,38 @@ e = launch_pdl(reduce_parts_kernel, dim3(hblocks > 0 ? hblocks : 1), dim3(256), 
                       E, d, b_down, 0, static_cast<__nv_bfloat16 *>(out));
 }
 
+cudaError_t launch_tc_bwd_gemms(const BwdArgs &a, const void *dO, void *dZ, void *dX, uint32_t *status,
+                                uint64_t timeout_ns, int num_sms, cudaStream_t s) {
+    // dZ = (dO W_down[e]) * [H > 0]: tokens dO [rows][d] (K = d), W_down [E][d][d_ff] read MN-major
+    cudaError_t e = launch_tc2<EPI_BF16_MASK, 6, true>(dO, a.rows, a.W_down, a.E, a.d_ff, a.d, a.offsets, a.counts,
+                                                       dZ, a.d_ff, status, timeout_ns, num_sms, s, nullptr, 1, a.H);
+    if (e != cudaSuccess) return e;
+    // dX = dZ W_up[e]: tokens dZ [rows][d_ff] (K = d_ff), W_up [E][d_ff][d] read MN-major
+    e = launch_tc2<EPI_BF16, 6, true>(dZ, a.rows, a.W_up, a.E, a.d, a.d_ff, a.offsets, a.counts, dX, a.d, status,
+                                      timeout_ns, num_sms, s);
+    if (e != cudaSuccess) return e;
+    // dW_down[e] = dO^T H ([d][d_ff]), dW_up[e] = dZ^T X ([d_ff][d])
+    e = launch_wgrad(dO, a.H, a.rows, a.d, a.d_ff, a.offsets, a.counts, a.E, a.dW_down, status, timeout_ns, num_sms,
+                     s);
+    if (e != cudaSuccess) return e;
+    return launch_wgrad(dZ, a.x_gathered, a.rows, a.d_ff, a.d, a.offsets, a.counts, a.E, a.dW_up, status,
+                        timeout_ns, num_sms, s);
+}
+
 // Diagnostic: one CTA waits on a barrier that nothing completes.
 __global__ void wait_timeout_kernel(uint32_t *status, uint64_t timeout_ns) {
     __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t cta_status;
     const uint32_t b = smem_u32(&bar);
     if (threadIdx.x == 0) {
         mbar_init(b, 1);
         fence_barrier_init();
+        cta_status = 0u;
     }
     __syncthreads();
-    if (threadIdx.x == 0) mbar_wait_bounded(b, 0, status, timeout_ns, 9);
+    if (threadIdx.x == 0) mbar_wait_bounded(b, 0, &cta_status, timeout_ns, 9);
     __syncthreads();
+    if (threadIdx.x == 0) publish_status(status, cta_status);
 }
 
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s) {

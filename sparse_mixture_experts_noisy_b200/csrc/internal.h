@@ -28,8 +28,10 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-// Router (route.cu).  status (nullable) is zeroed by the first block.  w3
-// (nullable): route_tc_w3_bytes(d, E) of scratch for the tensor-core router.
+// Router (route.cu).  status (nullable): the status word the tensor-core
+// router ORs a timeout into (never cleared here); null selects the library's
+// own per-device word (route_status_read_clear).  w3 (nullable):
+// route_tc_w3_bytes(d, E) of scratch for the tensor-core router.
 cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b_g,
                          const float *noise, float sigma, int64_t N, int d, int E, int k,
                          float *logits_out, int32_t *topk_idx, float *gates, uint32_t *status,
@@ -50,6 +52,9 @@ size_t route_tc_w3_bytes(int d, int E);
 cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, const float *noise, float sigma,
                             int64_t N, int d, int E, int k, float *logits_out, int32_t *topk_idx, float *gates,
                             uint32_t *status, uint64_t timeout_ns, void *w3, cudaStream_t s);
+// Reads and clears (on stream s, then synchronises it) the library's own status
+// word of router calls made without one, on the current device.
+cudaError_t route_status_read_clear(uint32_t *word, cudaStream_t s);
 
 // Dispatch (dispatch.cu).
 int64_t dispatch_blocks(int64_t N);
@@ -115,5 +120,38 @@ cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t 
                           TcPlan *plan_out, int act = 1, const float *b_up = nullptr,
                           const float *b_down = nullptr);
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
+
+// Backward (backward.cu, tensor-core GEMMs in gemm_tc.cu).  Pointers as in
+// moe_backward (include/moe.h); dt 1 = bf16 storage, 0 = fp32.
+struct BwdArgs {
+    const void *x;
+    int dt;
+    const float *W_g;
+    const void *W_up, *W_down;
+    int64_t N;
+    int d, E, d_ff, k;
+    int64_t rows;
+    const int32_t *topk;
+    const float *gates;
+    const int32_t *slot, *offsets, *counts;
+    const void *x_gathered, *H, *out_gathered, *dy;
+    void *dx;
+    float *dW_g, *db_g, *dW_up, *dW_down;
+};
+// Byte offsets inside the backward workspace (after the status word): the
+// gradient rows dO [rows][d], dZ [rows][d_ff], dX [rows][d] of the storage
+// type, ds [N][k] fp32, and the router-gradient chunk sums.
+struct BwdLayout {
+    size_t dO, dZ, dX, ds, part, total;
+};
+BwdLayout bwd_layout(const BwdArgs &a, int num_sms);
+cudaError_t launch_backward(const BwdArgs &a, void *ws, uint32_t *status, uint64_t timeout_ns, int num_sms,
+                            bool tensor_cores, cudaStream_t s);
+// The four expert GEMMs of the backward on the tensor cores (bf16):
+// dZ = (dO W_down[e]) * [H > 0], dX = dZ W_up[e] (CTA pairs, weights read
+// MN-major) and dW_down = dO^T H, dW_up = dZ^T X (K = the expert's rows).
+cudaError_t launch_tc_bwd_gemms(const BwdArgs &a, const void *dO, void *dZ, void *dX, uint32_t *status,
+                                uint64_t timeout_ns, int num_sms, cudaStream_t s);
+int backward_launches(const BwdArgs &a, bool tensor_cores);
 
 }  // namespace moe

@@ -104,7 +104,7 @@ route_tile_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
     float *s_sc = ws + kTileEC * kTileDC;                  // [kTileTok][E]
     float *pick_v = s_sc + static_cast<size_t>(kTileTok) * E + static_cast<size_t>(threadIdx.x >> 5) * 2 * k;
     int *pick_e = reinterpret_cast<int *>(pick_v + k);
-    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+    (void)status;  // no waits here, so nothing to report
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileTok + warp * kTileTPW;
     const int ntok = (t0 >= N) ? 0 : ((N - t0 < kTileTPW) ? static_cast<int>(N - t0) : kTileTPW);
@@ -261,7 +261,7 @@ route_block_kernel(const T *__restrict__ x, const float *__restrict__ W_g,
     float *sc = route_smem;            // [E]
     float *pick_v = sc + E;            // [k]
     int *pick_e = reinterpret_cast<int *>(pick_v + k);  // [k]
-    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
+    (void)status;  // no waits here, so nothing to report
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = blockIdx.x;
     const T *xr = x + t * static_cast<int64_t>(d);
@@ -371,7 +371,7 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
                          const float *noise, float sigma, int64_t N, int d, int E, int k,
                          float *logits_out, int32_t *topk_idx, float *gates, uint32_t *status,
                          cudaStream_t s, void *w3) {
-    if (N == 0) return status ? cudaMemsetAsync(status, 0, sizeof(uint32_t), s) : cudaSuccess;
+    if (N == 0) return cudaSuccess;
     const uintptr_t ax = reinterpret_cast<uintptr_t>(x), aw = reinterpret_cast<uintptr_t>(W_g);
     if (dt == 1 && route_tc_eligible(x, W_g, N, d, E, k))
         return launch_route_tc(x, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, status,

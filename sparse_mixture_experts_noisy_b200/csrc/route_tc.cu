@@ -58,7 +58,8 @@ constexpr int kRouteTcMaxK = 32;                   // pick scratch: k floats per
 constexpr size_t kRouteSmemBudget = 110 * 1024;    // per CTA: two CTAs fit on an SM
 constexpr size_t kRpSmemBudget = 225 * 1024;       // per CTA when one fills the SM
 
-// Status word for callers that pass none (moe_route): waits still need one.
+// Status word of calls that pass none (moe_route): one per device, read and
+// cleared by route_status_read_clear (moe_check_route_status).
 __device__ uint32_t g_route_status_scratch;
 
 struct RouteTcArgs {
@@ -72,7 +73,7 @@ struct RouteTcArgs {
     float *logits_out;
     int32_t *topk_idx;
     float *gates;
-    uint32_t *status;  // nullable: the kernel then uses a scratch word of its own
+    uint32_t *status;  // nullable: the kernel then reports into the library's own word
     uint64_t timeout_ns;
 };
 
@@ -390,6 +391,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 2];
     __shared__ uint32_t tmem_holder;
     __shared__ int epi_fail;
+    __shared__ uint32_t cta_status;  // this CTA's copy of the status word
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int stages = args.stages;
@@ -400,7 +402,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int kb0 = route_kb_begin(crank, S, kb_total), kb1 = route_kb_begin(crank + 1, S, kb_total);
     const int64_t t0 = static_cast<int64_t>(blockIdx.x / S) * kRM;
     const uint64_t tmo = args.timeout_ns;
-    uint32_t *status = args.status != nullptr ? args.status : &g_route_status_scratch;
+    uint32_t *status = &cta_status;
 
     const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
@@ -420,6 +422,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         mbar_init(drain, 1);
         fence_barrier_init();
         epi_fail = 0;
+        cta_status = 0u;
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_x);
@@ -437,7 +440,6 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     pdl_trigger();
     const uint32_t tmem_base = tmem_holder;
     pdl_wait();
-    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -606,6 +608,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
     }
     cluster_sync();  // no CTA leaves while another may still read its table
+    if (threadIdx.x == 0)
+        publish_status(args.status != nullptr ? args.status : &g_route_status_scratch, cta_status);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
@@ -642,6 +646,7 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     extern __shared__ uint8_t dyn_smem[];
     __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 5];
     __shared__ uint32_t tmem_holder;
+    __shared__ uint32_t cta_status;  // this CTA's copy of the status word
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int stages = args.stages;
@@ -650,7 +655,7 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     const int S = args.splits;
     const int64_t tiles = (args.N + kRM - 1) / kRM;
     const uint64_t tmo = args.timeout_ns;
-    uint32_t *status = args.status != nullptr ? args.status : &g_route_status_scratch;
+    uint32_t *status = &cta_status;
 
     const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
@@ -673,6 +678,7 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         }
         mbar_init(drain, 1);
         fence_barrier_init();
+        cta_status = 0u;
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_x);
@@ -688,7 +694,6 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     pdl_trigger();  // after the tensor memory is held (see the clustered form)
     const uint32_t tmem_base = tmem_holder;
     pdl_wait();
-    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -870,6 +875,8 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0)
+        publish_status(args.status != nullptr ? args.status : &g_route_status_scratch, cta_status);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
@@ -1034,6 +1041,16 @@ cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, c
     const bool persistent = tiles * a.splits >= 2 * static_cast<int64_t>(sms) && route_tcp_enabled();
     return w3 != nullptr ? launch_upt<true>(upt, persistent, tm, tw, a, tiles, sms, s)
                          : launch_upt<false>(upt, persistent, tm, tw, a, tiles, sms, s);
+}
+
+cudaError_t route_status_read_clear(uint32_t *word, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(word, g_route_status_scratch, sizeof(uint32_t), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    const uint32_t zero = 0u;
+    e = cudaMemcpyToSymbolAsync(g_route_status_scratch, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(s);
 }
 
 }  // namespace moe

@@ -21,9 +21,11 @@ ACT_RELU, ACT_GELU = 1, 2
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
-EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
+EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_route_ex", "moe_check_route_status",
+           "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_shard_workspace_size", "moe_shard_count", "moe_shard_base", "moe_shard_dispatch",
-           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_combine",
+           "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_expert_ffn_train",
+           "moe_backward_workspace_size", "moe_backward", "moe_combine",
            "moe_load_stats_workspace_size", "moe_load_stats",
            "moe_workspace_size", "moe_forward", "moe_forward_ex", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
@@ -54,6 +56,8 @@ def load_library(path: str = LIB_PATH):
             "moe_capacity": (I64, [I64, I, I, D]),
             "moe_gathered_rows": (I64, [I64, I, I, D]),
             "moe_route": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P]),
+            "moe_route_ex": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P, P]),
+            "moe_check_route_status": (I, [P, ctypes.POINTER(U32)]),
             "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
             "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
             "moe_dispatch_noalloc": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P]),
@@ -66,6 +70,10 @@ def load_library(path: str = LIB_PATH):
             "moe_expert_ffn_workspace_size": (SZ, [I64, I, I, I, I]),
             "moe_expert_ffn": (I, [P, P, P, P, P, I, I64, I, I, I, P, P, SZ, P]),
             "moe_expert_ffn_ex": (I, [P, P, P, P, P, I, I64, I, I, I, I, P, P, P, P, SZ, P]),
+            "moe_expert_ffn_train": (I, [P, P, P, P, P, I, I64, I, I, I, P, P, P, SZ, P]),
+            "moe_backward_workspace_size": (SZ, [I64, I, I, I, I, I64, I]),
+            "moe_backward": (I, [P, I, P, P, P, I64, I, I, I, I, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                 P, SZ, P]),
             "moe_combine": (I, [P, P, P, P, P, I, I64, I, I, P, P]),
             "moe_workspace_size": (SZ, [I64, I, I, I, I, D, I]),
             "moe_forward": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, P, P, P, P, P, P, P, SZ, P]),
@@ -132,8 +140,18 @@ def num_sms() -> int:
     return int(load_library().moe_num_sms())
 
 
-def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stream=None):
-    """-> (topk_idx [N,k] int32, gates [N,k] fp32, logits [N,E] fp32 or None)."""
+def new_workspace(nbytes, device):
+    """A device workspace whose status word (first 4 bytes) starts at zero."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stream=None, status=None):
+    """-> (topk_idx [N,k] int32, gates [N,k] fp32, logits [N,E] fp32 or None).
+    status (a workspace, nullable): where a router timeout is recorded (read it
+    with check_status); None records into the library's own word
+    (check_route_status)."""
     L = load_library()
     for t, n in ((x, "x"), (W_g, "W_g"), (b_g, "b_g"), (noise, "noise")):
         _cuda(t, n)
@@ -143,9 +161,17 @@ def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stre
     topk = torch.empty((N, k), dtype=torch.int32, device=dev)
     gates = torch.empty((N, k), dtype=torch.float32, device=dev)
     logits = torch.empty((N, E), dtype=torch.float32, device=dev) if want_logits else None
-    _check(L.moe_route(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, k,
-                       _p(logits), _p(topk), _p(gates), _stream(stream)))
+    _cuda(status, "status")
+    _check(L.moe_route_ex(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, k,
+                          _p(logits), _p(topk), _p(gates), _p(status), _stream(stream)))
     return topk, gates, logits
+
+
+def check_route_status(stream=None):
+    """Read/clear the library's router status word (moe_route without one) -> (code, raw word)."""
+    word = ctypes.c_uint32(0)
+    code = load_library().moe_check_route_status(_stream(stream), ctypes.byref(word))
+    return int(code), int(word.value)
 
 
 def moe_dispatch(topk_idx, x, E, cf, stream=None):
@@ -249,7 +275,7 @@ def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=No
     dt = _dt(x_gathered)
     wsb = L.moe_expert_ffn_workspace_size(rows, d, E, d_ff, dt)
     if ws is None:
-        ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=x_gathered.device)
+        ws = new_workspace(wsb, x_gathered.device)
     if out is None:
         out = torch.empty((rows, d), dtype=x_gathered.dtype, device=x_gathered.device)
     for t, n in ((b_up, "b_up"), (b_down, "b_down")):
@@ -257,6 +283,54 @@ def moe_expert_ffn(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=No
     _check(L.moe_expert_ffn_ex(_p(x_gathered), _p(offsets), _p(counts), _p(W_up), _p(W_down), dt, rows, d,
                                d_ff, E, int(act), _p(b_up), _p(b_down), _p(out), _p(ws), ws.numel(),
                                _stream(stream)))
+    return out
+
+
+def moe_expert_ffn_train(x_gathered, offsets, counts, W_up, W_down, stream=None, ws=None):
+    """Expert FFN that keeps the hidden activations for the backward.
+    -> (out_gathered [rows, d], H [rows, d_ff])."""
+    L = load_library()
+    for t, n in ((x_gathered, "x_gathered"), (offsets, "offsets"), (counts, "counts"), (W_up, "W_up"),
+                 (W_down, "W_down")):
+        _cuda(t, n)
+    rows, d = x_gathered.shape
+    E, d_ff, _ = W_up.shape
+    dt = _dt(x_gathered)
+    if ws is None:
+        ws = new_workspace(L.moe_expert_ffn_workspace_size(rows, d, E, d_ff, dt), x_gathered.device)
+    out = torch.empty((rows, d), dtype=x_gathered.dtype, device=x_gathered.device)
+    H = torch.empty((rows, d_ff), dtype=x_gathered.dtype, device=x_gathered.device)
+    _check(L.moe_expert_ffn_train(_p(x_gathered), _p(offsets), _p(counts), _p(W_up), _p(W_down), dt, rows, d, d_ff,
+                                  E, _p(out), _p(H), _p(ws), ws.numel(), _stream(stream)))
+    return out, H
+
+
+def moe_backward(x, W_g, W_up, W_down, k, topk_idx, gates, slot, offsets, counts, x_gathered, H, out_gathered, dy,
+                 stream=None, ws=None):
+    """Gradients of sum(dy * y) for the routing of a staged forward.
+    -> dict(dx [N, d] of x's dtype, dW_g [E, d], db_g [E], dW_up [E, d_ff, d], dW_down [E, d, d_ff] fp32)."""
+    L = load_library()
+    for t, n in ((x, "x"), (W_g, "W_g"), (W_up, "W_up"), (W_down, "W_down"), (topk_idx, "topk_idx"),
+                 (gates, "gates"), (slot, "slot"), (offsets, "offsets"), (counts, "counts"),
+                 (x_gathered, "x_gathered"), (H, "H"), (out_gathered, "out_gathered"), (dy, "dy")):
+        _cuda(t, n)
+    N, d = x.shape
+    E, d_ff, _ = W_up.shape
+    rows = x_gathered.shape[0]
+    dt = _dt(x)
+    dev = x.device
+    if ws is None:
+        ws = new_workspace(L.moe_backward_workspace_size(N, d, E, d_ff, k, rows, dt), dev)
+    out = dict(dx=torch.empty((N, d), dtype=x.dtype, device=dev),
+               dW_g=torch.empty((E, d), dtype=torch.float32, device=dev),
+               db_g=torch.empty(E, dtype=torch.float32, device=dev),
+               dW_up=torch.empty((E, d_ff, d), dtype=torch.float32, device=dev),
+               dW_down=torch.empty((E, d, d_ff), dtype=torch.float32, device=dev))
+    _check(L.moe_backward(_p(x), dt, _p(W_g), _p(W_up), _p(W_down), N, d, E, d_ff, k, rows, _p(topk_idx),
+                          _p(gates), _p(slot), _p(offsets), _p(counts), _p(x_gathered), _p(H), _p(out_gathered),
+                          _p(dy), _p(out["dx"]), _p(out["dW_g"]), _p(out["db_g"]), _p(out["dW_up"]),
+                          _p(out["dW_down"]), _p(ws), ws.numel(), _stream(stream)))
+    out["ws"] = ws
     return out
 
 
@@ -314,7 +388,7 @@ def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=
     if wsb == 0:
         raise MoeError(1, "invalid layer arguments")
     if ws is None:
-        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        ws = new_workspace(wsb, dev)
     if y is None:
         y = torch.empty((N, d), dtype=x.dtype, device=dev)
     inter = None
@@ -362,7 +436,7 @@ class MoELayer:
     def _reserve(self, N, dtype):
         need = workspace_size(N, self.d, self.E, self.d_ff, self.k, self.cf, dtype)
         if self._ws is None or self._ws.numel() < need:
-            self._ws = torch.empty(need, dtype=torch.uint8, device=self.W_up.device)
+            self._ws = new_workspace(need, self.W_up.device)
         self._ws_tokens = N
 
     @property

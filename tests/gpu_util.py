@@ -97,3 +97,66 @@ def check_routing(case: Case, inter, logits_tol=None):
     assert np.array_equal(inter["slot"].cpu().numpy(), slot), "slots differ from the oracle"
     assert np.array_equal(inter["counts"].cpu().numpy(), counts), "counts differ from the oracle"
     return lg, idx, g, slot, counts
+
+
+# ---------------------------------------------------------------------------
+# Per-element check of the bf16 path.
+#
+# The max-normalised error above cannot see a wrong element that is small
+# next to the row maximum.  This check bounds every element by the rounding
+# the bf16 path performs, as a statistical model: the hidden activations H are
+# rounded to bf16 after the activation, each expert output O to bf16 (in the
+# prefill plan), and y to bf16; the fp32 accumulations are far finer and are
+# covered by a tiny absolute floor.  A round-to-nearest bf16 error of a value v
+# is at most 2^-8 |v| and its variance at most (2^-8)^2 v^2 / 3 (a uniform
+# error on half an ulp), so for element i of token t
+#
+#   var_i = (2^-16 / 3) * ( sum_j g_j^2 [ sum_f W_down[e_j][i, f]^2 H_jf^2 + O_ji^2 ] + y_i^2 )
+#
+# and the test requires |y_i - y_oracle_i| <= Z_MAX * sqrt(var_i) + floor.  The
+# model only over-estimates the variance, and with Z_MAX = 8 a correct
+# element fails with a probability far below 1e-12.  An element that is wrong
+# by more than a few percent of the row's typical magnitude sits hundreds of
+# sigmas out, whatever its own size.
+U_BF16 = 2.0 ** -8
+Z_MAX = 8.0
+
+
+def bf16_error_sigma(inp, wl, tokens, idx, g, slot, y_ref):
+    """sigma_i of the model above for the rows `tokens` (y_ref: the oracle's
+    float64 rows for those tokens, same order).  Uses ReLU experts without
+    biases, the layer the parity tests run."""
+    tokens = np.asarray(tokens)
+    x = values(inp.x)[tokens].astype(np.float32)
+    var = np.zeros((len(tokens), wl.d))
+    u2 = U_BF16 * U_BF16 / 3.0
+    idx_t, slot_t, g_t = idx[tokens], slot[tokens], g[tokens].astype(np.float64)
+    for e in range(wl.E):
+        sel_t, sel_j = np.nonzero((idx_t == e) & (slot_t >= 0))
+        if len(sel_t) == 0:
+            continue
+        wu = bf16_bits_to_f32(inp.W_up[e]) if inp.W_up.dtype == np.uint16 else inp.W_up[e].astype(np.float32)
+        wd = bf16_bits_to_f32(inp.W_down[e]) if inp.W_down.dtype == np.uint16 else inp.W_down[e].astype(np.float32)
+        H = np.maximum(x[sel_t] @ wu.T, 0.0)
+        O = (H @ wd.T).astype(np.float64)
+        S2 = ((H * H) @ (wd * wd).T).astype(np.float64)
+        gg = g_t[sel_t, sel_j] ** 2
+        np.add.at(var, sel_t, gg[:, None] * u2 * (S2 + O * O))
+    var += u2 * y_ref * y_ref
+    return np.sqrt(var)
+
+
+def check_elementwise_bf16(y: np.ndarray, y_ref: np.ndarray, sigma: np.ndarray, what: str = "") -> float:
+    """Every element within Z_MAX sigma of the oracle (plus a floor of 2^-20 of
+    the largest |y_ref| for the fp32 accumulations).  Returns the largest
+    |error| / sigma seen."""
+    floor = 2.0 ** -20 * (float(np.max(np.abs(y_ref))) if y_ref.size else 0.0)
+    err = np.abs(y - y_ref)
+    bad = err > Z_MAX * sigma + floor
+    ratio = float(np.max(err / np.maximum(sigma, 1e-300))) if y.size else 0.0
+    if np.any(bad):
+        t, i = np.unravel_index(int(np.argmax(np.where(bad, err / np.maximum(sigma, 1e-300), 0))), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} elements outside {Z_MAX} sigma of the rounding model; "
+                             f"worst row {t} col {i}: got {y[t, i]:.6g}, oracle {y_ref[t, i]:.6g}, "
+                             f"sigma {sigma[t, i]:.3g}")
+    return ratio

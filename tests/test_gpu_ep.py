@@ -4,7 +4,10 @@ table and the all-to-alls by copying each rank's send views into the
 receivers' buffers, which is all the collectives do.  The result must match
 the same batch run as one unsharded call: the same slots and drop set bit for
 bit, and the output within the bf16 tolerance (a rank's expert calls see
-fewer rows, which can choose a different tile plan)."""
+fewer rows, which can choose a different tile plan).  It is also checked
+against the oracle on the whole batch, replaying the GPU's fp32 logits:
+top-k, drop set and queue order bit for bit, a sample of token outputs within
+the bf16 tolerance and the per-element rounding model."""
 import numpy as np
 import pytest
 import torch
@@ -12,6 +15,7 @@ import torch
 from sparse_mixture_experts_noisy_b200 import ep, moe
 from sparse_mixture_experts_noisy_b200.synth import WORKLOADS
 from tests.gpu_util import Case, TOL, rel_err, require_gpu, to_host_bits, values
+from tests.test_gpu_shard import check_shards_against_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -69,3 +73,7 @@ def test_expert_parallel_matches_unsharded(name):
     assert np.array_equal(kept_tot, d_r["counts"].cpu().numpy())
     err = rel_err(values(to_host_bits(y)), values(to_host_bits(y_ref)))
     assert err <= TOL[wl.dtype], f"{name}: {err:.3g}"
+    lg = torch.cat([moe.moe_route(xs[g], case.W_g, k, b_g=case.b_g, noise=ns[g], sigma=wl.sigma)[2]
+                    for g in range(G)]).cpu().numpy()
+    check_shards_against_oracle(case, cuts, [s["topk"].cpu().numpy() for s in st],
+                                [s["dispatch"]["slot"].cpu().numpy() for s in st], y, lg)
