@@ -47,6 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the secondary decode measurement")
     ap.add_argument("--only", action="store_true", help="measure only --workload (no secondary workloads)")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward measurement")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (small cases for profiling); implies --only")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -465,10 +466,61 @@ def measure_workload(wl, inp_dev, steps, warmup, dist, dev, torch, moe, peaks, p
                               {"frac_of_sustained": fl / ffn_sec / 1e12 / peaks["bf16_tflops_sustained"],
                                "algorithmic_flops": fl, "kept_rows": R, "ms_per_call": ffn_sec * 1e3,
                                "whole_layer_frac": fl / step_s / 1e12 / peaks["bf16_tflops"]})
+    router = None
+    if wl.dtype == "bf16":
+        # the router alone (moe_forward's pre-split path), against the copy bandwidth
+        rws = moe.route_workspace(wl.d, wl.E, dev)
+        x, W_g, b_g, noise = inp_dev[:4]
+        rrun = lambda: moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma,  # noqa: E731
+                                     want_logits=False, status=rws)
+        for _ in range(3):
+            rrun()
+        torch.cuda.synchronize()
+        rsec = time_steps(rrun, max(20, min(steps, 200)), torch, flush) / max(20, min(steps, 200))
+        rbytes = wl.N * wl.d * elem + (wl.N * wl.E * 4 if noise is not None else 0) + wl.N * wl.k * 8
+        router = {"us_per_call": rsec * 1e6, "algorithmic_bytes": rbytes, "gbs": rbytes / rsec / 1e9,
+                  "frac": rbytes / rsec / 1e9 / peaks["hbm_gbs"], "peak_source": peak_src + " (copy)"}
     out = {"workload": wl.name, "value": agg["value"], "unit": UNIT, "ms_per_step": agg["ms_per_step"],
-           "steps": steps, "config": workload_config(wl), "roofline": roof, "clocks": clocks,
+           "steps": steps, "config": workload_config(wl), "roofline": roof, "clocks": clocks, "router": router,
            "gpu_launches": moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) * steps}
     return out, graphed
+
+
+def measure_backward(wl, inp_dev, steps, dist, dev, torch, moe, peaks, peak_src, seed):
+    """The backward of the layer (moe_backward) for the routing of one staged
+    forward, on the forward's kept activations: its four expert GEMMs are
+    2 R d d_ff flops each.  Timed with CUDA events over back-to-back calls."""
+    from sparse_mixture_experts_noisy_b200.synth import f32_to_bf16_bits, normal_f32
+    x, W_g, b_g, noise, W_up, W_down = inp_dev
+    topk, gates, _ = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma, want_logits=False)
+    dsp = moe.moe_dispatch(topk, x, wl.E, wl.cf)
+    out, H = moe.moe_expert_ffn_train(dsp["x_gathered"], dsp["offsets"], dsp["counts"], W_up, W_down)
+    dyh = normal_f32(seed + 5, (wl.N, wl.d), 1.0)
+    dy = to_dev(f32_to_bf16_bits(dyh) if wl.dtype == "bf16" else dyh, torch)
+    args = (x, W_g, W_up, W_down, wl.k, topk, gates, dsp["slot"], dsp["offsets"], dsp["counts"], dsp["x_gathered"], H,
+            out, dy)
+    g = moe.moe_backward(*args)
+    ws = g["ws"]
+    run = lambda: moe.moe_backward(*args, ws=ws)  # noqa: E731
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = ClockSampler(dev)
+    with clk:
+        sec = time_steps(run, steps, torch)
+    code, word = moe.check_status(ws)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code} (0x{word:08x}) after the backward timing")
+    sec = dist.max(sec, device=dev)
+    R = int(dsp["counts"].sum().item())
+    fl = 2.0 * ffn_flops(R, wl.d, wl.d_ff)
+    return {"workload": wl.name, "what": "moe_backward: dx, dW_g, db_g, dW_up, dW_down for one routed batch",
+            "value": wl.N * dist.world * steps / sec, "unit": UNIT, "ms_per_step": 1e3 * sec / steps, "steps": steps,
+            "roofline": roofline_entry("tensor", fl / (sec / steps) / 1e12, peaks["bf16_tflops"], "TFLOP/s", None,
+                                       "whole backward (four expert GEMMs on the tensor cores + per-token kernels)",
+                                       peak_src + " burst", {"algorithmic_flops": fl, "kept_rows": R}),
+            "clocks": clk.summary()}
 
 
 # timed steps of the secondary workloads, whatever --steps is: enough that the
@@ -519,6 +571,11 @@ def run_ours(args):
             "gpu_launches": main["gpu_launches"],
             "clocks": main["clocks"]}
     del graphed
+
+    if wl.dtype == "bf16" and not args.no_backward:
+        line["backward"] = measure_backward(wl, inp_dev, max(10, min(args.steps, 50)), dist, dev, torch, moe, peaks,
+                                            peak_src, args.seed)
+        torch.cuda.empty_cache()
 
     # every other workload, each with its own timed region, roofline and clocks
     if args.workload == "mixtral" and not args.only:

@@ -118,14 +118,19 @@ MOE_API moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, cons
                      const float *noise, float sigma, int64_t N, int d, int E, int k,
                      float *logits_out, int32_t *topk_idx, float *gates, void *stream);
 
-/* moe_route with the caller's status word: `status` (device, 16-byte aligned,
- * at least 4 bytes, zero before first use; NULL selects the library's word as
- * in moe_route) receives the error bits, and moe_check_status(status, ...)
- * reads and clears it.  A workspace of moe_forward can serve: its status word
- * is its first 4 bytes. */
+/* Workspace bytes with which moe_route_ex takes moe_forward's router path. */
+MOE_API size_t moe_route_workspace_size(int d, int E);
+
+/* moe_route with a caller workspace.  ws (device, 16-byte aligned, nullable):
+ *  - NULL: exactly moe_route (the library's status word);
+ *  - ws_bytes >= 256: its first 4 bytes are the status word (zero before first
+ *    use), read and cleared by moe_check_status(ws, ...);
+ *  - ws_bytes >= moe_route_workspace_size(d, E), bf16 tokens: the router
+ *    weights are also split into ws first and read from there (moe_forward's
+ *    router: on many tokens the CTA-pair form).  Same results either way. */
 MOE_API moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                                 const float *noise, float sigma, int64_t N, int d, int E, int k,
-                                float *logits_out, int32_t *topk_idx, float *gates, void *status,
+                                float *logits_out, int32_t *topk_idx, float *gates, void *ws, size_t ws_bytes,
                                 void *stream);
 
 /* Synchronises `stream` after reading and clearing (on that stream) the

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 
@@ -85,8 +86,34 @@ size_t ffn_ws_bytes(int64_t rows, int d, int E, int d_ff, moe_dtype dt) {
 }
 
 struct FwdLayout {
-    size_t status, topk, gates, slot, counts, offsets, dws, w3, xg, og, ffn, total;
+    size_t status, topk, gates, slot, counts, offsets, dws, w3, xg, og, ffn, fused, total;
 };
+
+// Small batches run the whole layer as one cooperative kernel when the shape
+// allows (decode_fused.cu); MOE_FUSED_DECODE=0 keeps the separate kernels.
+bool fused_decode_enabled() {
+    static const bool on = [] {
+        const char *v = getenv("MOE_FUSED_DECODE");
+        return v == nullptr || atoi(v) != 0;
+    }();
+    return on;
+}
+
+// Whether moe_forward takes the fused small-batch kernel (pointers nullable:
+// then their alignment is assumed).
+bool use_fused_decode(const void *x, const float *W_g, int64_t N, int d, int E, int d_ff, int k, int64_t rows,
+                      moe_dtype dt, int act, const float *b_up, const float *b_down) {
+    if (!fused_decode_enabled() || dt != MOE_BF16 || !use_tensor_cores(dt, d, d_ff) || act != MOE_ACT_RELU ||
+        b_up != nullptr || b_down != nullptr)
+        return false;
+    const int sms = num_sms_current();
+    const moe::TcPlan p = moe::plan_tc_ffn(rows, d, d_ff, E, sms);
+    if (!p.decode || p.splits_up < 2) return false;
+    static const uint64_t kAligned[2] = {0, 0};
+    const void *xa = x ? x : kAligned;
+    const float *wa = W_g ? W_g : reinterpret_cast<const float *>(kAligned);
+    return moe::decode_fused_eligible(xa, wa, N, d, E, d_ff, k, rows, sms);
+}
 
 FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows, moe_dtype dt) {
     using moe::align_up;
@@ -104,6 +131,7 @@ FwdLayout forward_layout(int64_t N, int d, int E, int d_ff, int k, int64_t rows,
     L.xg = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
     L.og = o; o += align_up(static_cast<size_t>(rows) * d * elem_bytes(dt), 256);
     L.ffn = o; o += ffn_ws_bytes(rows, d, E, d_ff, dt);
+    L.fused = o; o += (N <= 64 && dt == MOE_BF16) ? moe::decode_fused_scratch_bytes(N, d, E) : 0;
     L.total = o;
     return L;
 }
@@ -223,9 +251,15 @@ int64_t moe_gathered_rows(int64_t N, int E, int k, double cf) {
     return rows_for(N, E, k, C);
 }
 
+size_t moe_route_workspace_size(int d, int E) {
+    if (d < 1 || E < 1 || E > 256) return 0;
+    return moe::kStatusBytes + moe::route_tc_w3_bytes(d, E);
+}
+
 moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                         const float *noise, float sigma, int64_t N, int d, int E, int k,
-                        float *logits_out, int32_t *topk_idx, float *gates, void *status, void *stream) {
+                        float *logits_out, int32_t *topk_idx, float *gates, void *ws, size_t ws_bytes,
+                        void *stream) {
     moe_status st = check_shape(N, d, E, k, dt);
     if (st != MOE_OK) return st;
     if (N > 0) {
@@ -237,11 +271,19 @@ moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const flo
         OPTIONAL_PTR(noise, "noise");
         OPTIONAL_PTR(logits_out, "logits_out");
     }
-    OPTIONAL_PTR(status, "status");
+    OPTIONAL_PTR(ws, "ws");
+    if (ws != nullptr && ws_bytes < static_cast<size_t>(moe::kStatusBytes))
+        return fail(MOE_ERR_WORKSPACE, "router workspace needs at least %d bytes (got %zu)", moe::kStatusBytes,
+                    ws_bytes);
     if (!std::isfinite(sigma)) return fail(MOE_ERR_INVALID_ARG, "sigma must be finite");
+    // a workspace large enough for the split router weights: the pre-split path of moe_forward
+    const size_t w3 = moe::route_tc_w3_bytes(d, E);
+    void *w3p = (ws != nullptr && dt == MOE_BF16 && w3 > 0 && ws_bytes >= moe::kStatusBytes + w3)
+                    ? static_cast<void *>(static_cast<uint8_t *>(ws) + moe::kStatusBytes)
+                    : nullptr;
     cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
-                                      logits_out, topk_idx, gates, static_cast<uint32_t *>(status),
-                                      static_cast<cudaStream_t>(stream));
+                                      logits_out, topk_idx, gates, static_cast<uint32_t *>(ws),
+                                      static_cast<cudaStream_t>(stream), w3p);
     if (e != cudaSuccess) return cuda_fail(e, "router launch");
     return MOE_OK;
 }
@@ -249,7 +291,7 @@ moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const flo
 moe_status moe_route(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                      const float *noise, float sigma, int64_t N, int d, int E, int k,
                      float *logits_out, int32_t *topk_idx, float *gates, void *stream) {
-    return moe_route_ex(x, dt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, nullptr, stream);
+    return moe_route_ex(x, dt, W_g, b_g, noise, sigma, N, d, E, k, logits_out, topk_idx, gates, nullptr, 0, stream);
 }
 
 moe_status moe_check_route_status(void *stream, uint32_t *detail) {
@@ -618,6 +660,21 @@ moe_status moe_forward_ex(const void *x, moe_dtype dt, const float *W_g, const f
     void *xg = w + L.xg;
     void *og = w + L.og;
 
+    if (N > 0 && L.total > L.fused &&
+        use_fused_decode(x, W_g, N, d, E, d_ff, k, rows, dt, activation, b_up, b_down)) {
+        const int sms = num_sms_current();
+        const moe::TcPlan p = moe::plan_tc_ffn(rows, d, d_ff, E, sms);
+        uint8_t *f = w + L.ffn;
+        float *parts_dn = reinterpret_cast<float *>(f + moe::align_up(static_cast<size_t>(rows) * d_ff * 2, 256));
+        float *parts_up = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(parts_dn) +
+                                                    moe::align_up(static_cast<size_t>(p.splits_down) * rows * d * 4, 256));
+        cudaError_t e = moe::launch_decode_fused(x, W_g, b_g, noise, sigma, N, d, E, d_ff, k, C, W_up, W_down, y,
+                                                 logits_out, topk, gates, slot, counts, offsets, xg, rows, f, parts_dn,
+                                                 parts_up, p.splits_up, p.splits_down, w + L.fused, status,
+                                                 kWaitTimeoutNs, sms, s);
+        if (e != cudaSuccess) return cuda_fail(e, "fused small-batch layer launch");
+        return MOE_OK;
+    }
     void *w3 = (L.xg > L.w3) ? static_cast<void *>(w + L.w3) : nullptr;
     cudaError_t e = moe::launch_route(x, dt == MOE_BF16 ? 1 : 0, W_g, b_g, noise, sigma, N, d, E, k,
                                       logits_out, topk, gates, status, s, w3);
@@ -657,6 +714,9 @@ moe_status moe_forward(const void *x, moe_dtype dt, const float *W_g, const floa
 int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt) {
     if (check_shape(N, d, E, k, dt) != MOE_OK || d_ff < 1 || moe_capacity(N, E, k, cf) < 0) return -1;
     if (N == 0) return 0;
+    if (use_fused_decode(nullptr, nullptr, N, d, E, d_ff, k, rows_for(N, E, k, moe_capacity(N, E, k, cf)), dt,
+                         MOE_ACT_RELU, nullptr, nullptr))
+        return 1;
     int ffn = 2;
     if (use_tensor_cores(dt, d, d_ff)) {
         const int64_t rows = rows_for(N, E, k, moe_capacity(N, E, k, cf));

@@ -62,9 +62,6 @@ struct TcArgs {
     uint64_t timeout_ns;
     const float *bias;  // [E][Nw] fp32 or null: added to every output row of expert e
     int act;            // EPI_BF16_ACT: 1 = ReLU, 2 = GELU (x * Phi(x))
-    int group_m;        // pair tiles: M tiles per raster group (0 = all of the expert's)
-    int l2_hint;        // pair tiles: 0 both operands evict_normal; 1 token rows evict_last;
-                        // 2 token rows evict_last, weights evict_first
     const __nv_bfloat16 *mask;  // EPI_BF16_MASK: [rows][Nw], same layout as out
 };
 
@@ -510,21 +507,12 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
         int r = u - pre_s[lo];
         const int split = r % splits;
         r /= splits;
-        // Raster: the expert's M tiles in groups of at most group_m (balanced);
-        // inside a group M tiles fastest, then N tiles.  Units in flight at
-        // one time then share a few token-row tiles and a few weight tiles.
+        // M tiles fastest: a wave of units shares the expert's token rows and a
+        // few weight tiles (grouped M tiles and L2 eviction hints measured
+        // slower on the Mixtral shape)
         const int mt = (cnt_s[lo] + BT - 1) / BT;
-        const int nt = (Nw + BT - 1) / BT;
-        const int G = (args.group_m > 0 && args.group_m < mt) ? args.group_m : mt;
-        const int ng = (mt + G - 1) / G;
-        const int q = r / nt;  // group i holds units [m0(i) * nt, m0(i + 1) * nt)
-        int gi = static_cast<int>(static_cast<int64_t>(q) * ng / mt);
-        while (gi > 0 && gi * mt / ng > q) --gi;
-        while ((gi + 1) * mt / ng <= q) ++gi;
-        const int m0 = gi * mt / ng, gs = (gi + 1) * mt / ng - m0;
-        const int rr = r - m0 * nt;
-        tok0 = (m0 + rr % gs) * BT;
-        w0 = (rr / gs) * BT;
+        tok0 = (r % mt) * BT;
+        w0 = (r / mt) * BT;
         n_valid = min(BT, Nw - w0);
         kb0 = static_cast<int>(static_cast<int64_t>(split) * kb_total / splits);
         kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * kb_total / splits);
@@ -537,8 +525,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
             uint32_t phase = 0;
             bool ok = true;
             int issued = 0;
-            const uint64_t pol_tok = args.l2_hint >= 1 ? policy_evict_last() : policy_evict_normal();
-            const uint64_t pol_w = args.l2_hint >= 2 ? policy_evict_first() : policy_evict_normal();
+            const uint64_t pol = policy_evict_normal();
             for (int u = pair; u < total_units && ok; u += npairs) {
                 int e, tok0, w0, kb0, kb1, nv;
                 decode(u, e, tok0, w0, kb0, kb1, nv);
@@ -553,12 +540,12 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constan
                     const uint32_t fb = full0_lead + 8 * stage;
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
                     const int kx = kb * kBK;
-                    tma_load_2d_pair(sa, &tm_tok, fb, kx, tok_row, pol_tok);
+                    tma_load_2d_pair(sa, &tm_tok, fb, kx, tok_row, pol);
                     if constexpr (B_MN) {
-                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, w_row, kx, e, pol_w);
-                        tma_load_3d_pair(sa + A_BYTES + 8192u, &tm_w, fb, w_row + 64, kx, e, pol_w);
+                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, w_row, kx, e, pol);
+                        tma_load_3d_pair(sa + A_BYTES + 8192u, &tm_w, fb, w_row + 64, kx, e, pol);
                     } else {
-                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, kx, w_row, e, pol_w);
+                        tma_load_3d_pair(sa + A_BYTES, &tm_w, fb, kx, w_row, e, pol);
                     }
                     ++issued;
                     if (++stage == STAGES) {
@@ -723,30 +710,8 @@ cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, i
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act, 0, 0,
-             nullptr};
+    TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act, nullptr};
     return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, tm_tok, tm_w, a);
-}
-
-// Raster group and L2 policies of the pair tiles for a GEMM of depth K.
-// MOE_TC_GROUP_M and MOE_TC_L2HINT override them (for measurements).
-struct TcRaster {
-    int group_m, l2_hint;
-};
-TcRaster tc2_raster(int K) {
-    static const int env_group = [] {
-        const char *v = getenv("MOE_TC_GROUP_M");
-        return v ? atoi(v) : -1;
-    }();
-    static const int env_hint = [] {
-        const char *v = getenv("MOE_TC_L2HINT");
-        return v ? atoi(v) : -1;
-    }();
-    (void)K;
-    TcRaster r{0, 0};
-    if (env_group >= 0) r.group_m = env_group;
-    if (env_hint >= 0) r.l2_hint = env_hint;
-    return r;
 }
 
 template <int EPI, int STAGES, bool B_MN = false>
@@ -777,8 +742,7 @@ cudaError_t launch_tc2(const void *tok, int64_t tok_rows, const void *W, int E, 
         max_clusters < pairs)
         pairs = max_clusters;
     (void)cudaGetLastError();
-    const TcRaster rs = tc2_raster(K);
-    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns, bias, act, rs.group_m, rs.l2_hint,
+    TcArgs a{offsets, counts, E, Nw, K, 1, out, ldo, 0, status, timeout_ns, bias, act,
              static_cast<const __nv_bfloat16 *>(mask)};
     return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), smem, s, tm_tok, tm_w, a);
 }

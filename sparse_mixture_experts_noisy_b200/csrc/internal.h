@@ -121,6 +121,22 @@ cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t 
                           const float *b_down = nullptr);
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
 
+// The whole layer for at most 64 bf16 tokens in one cooperative launch
+// (decode_fused.cu).  Eligible shapes: E <= 16, k <= 32, the decode plan with
+// the up projection split over K (splits_up > 1), the tensor-core router.
+// scratch: decode_fused_scratch_bytes(); xg [rows][d], H [rows][d_ff],
+// parts_dn [s_dn][rows][d] and parts_up [s_up][rows][d_ff] as in the decode
+// plan.  Same results as the separate kernels, bit for bit.
+bool decode_fused_eligible(const void *x, const float *W_g, int64_t N, int d, int E, int d_ff, int k, int64_t rows,
+                           int num_sms);
+size_t decode_fused_scratch_bytes(int64_t N, int d, int E);
+cudaError_t launch_decode_fused(const void *x, const float *W_g, const float *b_g, const float *noise, float sigma,
+                                int64_t N, int d, int E, int d_ff, int k, int64_t C, const void *W_up,
+                                const void *W_down, void *y, float *logits_out, int32_t *topk, float *gates,
+                                int32_t *slot, int32_t *counts, int32_t *offsets, void *xg, int64_t rows, void *H,
+                                float *parts_dn, float *parts_up, int s_up, int s_dn, void *scratch,
+                                uint32_t *status, uint64_t timeout_ns, int num_sms, cudaStream_t s);
+
 // Backward (backward.cu, tensor-core GEMMs in gemm_tc.cu).  Pointers as in
 // moe_backward (include/moe.h); dt 1 = bf16 storage, 0 = fp32.
 struct BwdArgs {

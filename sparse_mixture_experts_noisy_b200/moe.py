@@ -21,7 +21,8 @@ ACT_RELU, ACT_GELU = 1, 2
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
                 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
-EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_route_ex", "moe_check_route_status",
+EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_route_ex", "moe_route_workspace_size",
+           "moe_check_route_status",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_dispatch_noalloc",
            "moe_shard_workspace_size", "moe_shard_count", "moe_shard_base", "moe_shard_dispatch",
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_expert_ffn_train",
@@ -56,7 +57,8 @@ def load_library(path: str = LIB_PATH):
             "moe_capacity": (I64, [I64, I, I, D]),
             "moe_gathered_rows": (I64, [I64, I, I, D]),
             "moe_route": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P]),
-            "moe_route_ex": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P, P]),
+            "moe_route_ex": (I, [P, I, P, P, P, F, I64, I, I, I, P, P, P, P, SZ, P]),
+            "moe_route_workspace_size": (SZ, [I, I]),
             "moe_check_route_status": (I, [P, ctypes.POINTER(U32)]),
             "moe_dispatch_workspace_size": (SZ, [I64, I, I]),
             "moe_dispatch": (I, [P, P, I, I64, I, I, I, D, P, P, P, P, P, SZ, P]),
@@ -147,11 +149,17 @@ def new_workspace(nbytes, device):
     return ws
 
 
+def route_workspace(d, E, device):
+    """A workspace with which moe_route takes moe_forward's router path."""
+    return new_workspace(load_library().moe_route_workspace_size(d, E), device)
+
+
 def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stream=None, status=None):
     """-> (topk_idx [N,k] int32, gates [N,k] fp32, logits [N,E] fp32 or None).
-    status (a workspace, nullable): where a router timeout is recorded (read it
-    with check_status); None records into the library's own word
-    (check_route_status)."""
+    status (a workspace, nullable): its first 4 bytes record a router timeout
+    (read them with check_status); None records into the library's own word
+    (check_route_status).  A workspace from route_workspace() also selects the
+    pre-split router of moe_forward."""
     L = load_library()
     for t, n in ((x, "x"), (W_g, "W_g"), (b_g, "b_g"), (noise, "noise")):
         _cuda(t, n)
@@ -163,7 +171,8 @@ def moe_route(x, W_g, k, b_g=None, noise=None, sigma=0.0, want_logits=True, stre
     logits = torch.empty((N, E), dtype=torch.float32, device=dev) if want_logits else None
     _cuda(status, "status")
     _check(L.moe_route_ex(_p(x), _dt(x), _p(W_g), _p(b_g), _p(noise), float(sigma), N, d, E, k,
-                          _p(logits), _p(topk), _p(gates), _p(status), _stream(stream)))
+                          _p(logits), _p(topk), _p(gates), _p(status), 0 if status is None else status.numel(),
+                          _stream(stream)))
     return topk, gates, logits
 
 

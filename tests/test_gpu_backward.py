@@ -35,8 +35,8 @@ CASES = {
     "decode_small": W["decode"].with_(N=64, d=512, d_ff=1024),
     # k = 1: the router gets no gradient
     "switch_k1": W["nano"].with_(N=700, d=128, d_ff=256, k=1, cf=1.0, wg_std=0.1),
-    # 16 experts for 20 tokens: some experts get no rows
-    "empty_experts": W["decode"].with_(N=20, d=256, d_ff=256, E=16, k=2),
+    # 16 experts for 6 tokens with 2 choices: at least 4 experts get no rows
+    "empty_experts": W["decode"].with_(N=6, d=256, d_ff=256, E=16, k=2),
     # fp32 storage: CUDA-core kernels throughout, drops and noise
     "f32_drops": Workload("f32_drops", F32, N=300, d=40, E=6, d_ff=50, k=3, sigma=0.5, cf=0.8,
                           w_std=0.3, wg_std=0.3),

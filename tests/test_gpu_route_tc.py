@@ -153,3 +153,32 @@ def test_router_batch_size_independent(name):
         assert torch.equal(l2.view(torch.int32), logits[sl].view(torch.int32)), (a, b)
         assert torch.equal(t2, topk[sl]), (a, b)
         assert torch.equal(g2.view(torch.int32), gates[sl].view(torch.int32)), (a, b)
+
+
+PRESPLIT_CASES = {
+    "e8_d4096": _wl("pe8", N=20000, d=4096, E=8, k=2, sigma=1.0, bias0=1.0),
+    "e24_odd_tiles": _wl("pe24", N=30001, d=512, E=24, k=3, sigma=0.5, wg_std=0.1),
+    "e64_fine": _wl("pe64", N=32768, d=2048, E=64, k=6, sigma=1.0),
+    "e80": _wl("pe80", N=40000, d=1024, E=80, k=4, sigma=0.5, wg_std=0.05, bias0=0.5),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PRESPLIT_CASES))
+def test_router_pre_split_matches_in_kernel_split(name):
+    """With a router workspace the weights are split once by a first pass and
+    read by TMA (moe_forward's router); without one, the router splits them
+    in-kernel.  Same bits, and the oracle's bar, on the persistent form with
+    balanced tiles (an odd tile count among them)."""
+    require_gpu()
+    wl = PRESPLIT_CASES[name]
+    inp = make_inputs(wl, seed=25, weights=False)
+    x, W_g, b_g, noise = to_dev(inp.x), to_dev(inp.W_g), to_dev(inp.b_g), to_dev(inp.noise)
+    ws = moe.route_workspace(wl.d, wl.E, x.device)
+    t1, g1, l1 = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma, status=ws)
+    t2, g2, l2 = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma)
+    torch.cuda.synchronize()
+    assert moe.check_status(ws) == (0, 0)
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
+    assert torch.equal(t1, t2)
+    assert torch.equal(g1.view(torch.int32), g2.view(torch.int32))
+    _check(wl, inp, t1.cpu().numpy(), g1.cpu().numpy(), l1.cpu().numpy())
