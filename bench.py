@@ -494,6 +494,21 @@ def measure_workload(wl, inp_dev, steps, warmup, dist, dev, torch, moe, peaks, p
     out = {"workload": wl.name, "value": agg["value"], "unit": UNIT, "ms_per_step": agg["ms_per_step"],
            "steps": steps, "config": workload_config(wl), "roofline": roof, "clocks": clocks, "router": router,
            "gpu_launches": moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) * steps}
+    if decode_plan and not moe.set_fused_small_batch(None):
+        # the same layer as one cooperative launch (opt-in), for comparison
+        moe.set_fused_small_batch(True)
+        try:
+            if moe.forward_launches(wl.N, wl.d, wl.E, wl.d_ff, wl.k, wl.cf, inp_dev[0].dtype) == 1:
+                fsteps = max(20, min(steps, 300))
+                fg, _, fsec, fclk = measure_layer(wl, inp_dev, fsteps, warmup, dist, torch, moe, flush_needed)
+                fsec = dist.max(fsec, device=dev)
+                del fg
+                out["single_launch"] = {"what": "decode_fused_kernel (moe_set_fused_small_batch(1))",
+                                        "ms_per_step": 1e3 * fsec / fsteps,
+                                        "value": wl.N * dist.world * fsteps / fsec, "unit": UNIT,
+                                        "steps": fsteps, "clocks": fclk}
+        finally:
+            moe.set_fused_small_batch(False)
     return out, graphed
 
 

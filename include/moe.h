@@ -127,7 +127,7 @@ MOE_API size_t moe_route_workspace_size(int d, int E);
  *    use), read and cleared by moe_check_status(ws, ...);
  *  - ws_bytes >= moe_route_workspace_size(d, E), bf16 tokens: the router
  *    weights are also split into ws first and read from there (moe_forward's
- *    router: on many tokens the CTA-pair form).  Same results either way. */
+ *    router: the persistent form on many tokens).  Same results either way. */
 MOE_API moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                                 const float *noise, float sigma, int64_t N, int d, int E, int k,
                                 float *logits_out, int32_t *topk_idx, float *gates, void *ws, size_t ws_bytes,
@@ -389,6 +389,16 @@ MOE_API moe_status moe_forward_ex(const void *x, moe_dtype dt, const float *W_g,
  * stream (0 for N = 0, -1 for invalid arguments).  Useful to size CUDA-graph
  * captures and to account for launches. */
 MOE_API int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, moe_dtype dt);
+
+/* Whether moe_forward runs batches of at most 64 bf16 tokens (E <= 16, ReLU
+ * experts without biases, the decode plan) as one cooperative kernel on every
+ * SM instead of the decode plan's separate kernels.  Both give identical
+ * bits.  on = 1 or 0 sets the choice for the process (calls already queued
+ * keep theirs); on < 0 only queries.  Returns the previous setting.  Default:
+ * off (on a B200 the separate kernels stream the expert weights faster), or on
+ * when the environment variable MOE_FUSED_DECODE is a nonzero number.  The
+ * workspace size does not depend on it; moe_forward_launches follows it. */
+MOE_API int moe_set_fused_small_batch(int on);
 
 /* ---------------------------------------------------------------- status */
 

@@ -1,5 +1,6 @@
 // The C ABI (include/moe.h): argument checks on the host, workspace carving,
 // and the launch sequence of the layer on one stream.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -89,14 +90,22 @@ struct FwdLayout {
     size_t status, topk, gates, slot, counts, offsets, dws, w3, xg, og, ffn, fused, total;
 };
 
-// Small batches run the whole layer as one cooperative kernel when the shape
-// allows (decode_fused.cu); MOE_FUSED_DECODE=0 keeps the separate kernels.
+// Whether small batches run the whole layer as one cooperative kernel when the
+// shape allows (decode_fused.cu).  Off unless MOE_FUSED_DECODE is a nonzero
+// number or moe_set_fused_small_batch(1) was called: on a B200 the separate
+// decode-plan kernels stream the weights faster.  -1: not read yet.
+std::atomic<int> g_fused_small_batch{-1};
+
 bool fused_decode_enabled() {
-    static const bool on = [] {
-        const char *v = getenv("MOE_FUSED_DECODE");
-        return v == nullptr || atoi(v) != 0;
-    }();
-    return on;
+    int v = g_fused_small_batch.load(std::memory_order_relaxed);
+    if (v < 0) {
+        const char *e = getenv("MOE_FUSED_DECODE");
+        int want = (e != nullptr && atoi(e) != 0) ? 1 : 0;
+        int expected = -1;
+        g_fused_small_batch.compare_exchange_strong(expected, want);
+        v = g_fused_small_batch.load(std::memory_order_relaxed);
+    }
+    return v != 0;
 }
 
 // Whether moe_forward takes the fused small-batch kernel (pointers nullable:
@@ -725,6 +734,12 @@ int moe_forward_launches(int64_t N, int d, int E, int d_ff, int k, double cf, mo
     // router (+ its weight split) + dispatch passes + expert FFN + combine
     const bool w3 = dt == MOE_BF16 && moe::route_tc_w3_bytes(d, E) > 0;
     return moe::route_launches(dt == MOE_BF16 ? 1 : 0, N, d, E, k, w3) + moe::dispatch_launches(N, E, k) + ffn + 1;
+}
+
+int moe_set_fused_small_batch(int on) {
+    const int prev = fused_decode_enabled() ? 1 : 0;
+    if (on >= 0) g_fused_small_batch.store(on != 0 ? 1 : 0, std::memory_order_relaxed);
+    return prev;
 }
 
 moe_status moe_check_status(void *ws, void *stream, uint32_t *detail) {

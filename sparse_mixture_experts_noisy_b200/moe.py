@@ -28,7 +28,8 @@ EXPORTS = ("moe_capacity", "moe_gathered_rows", "moe_route", "moe_route_ex", "mo
            "moe_expert_ffn_workspace_size", "moe_expert_ffn", "moe_expert_ffn_ex", "moe_expert_ffn_train",
            "moe_backward_workspace_size", "moe_backward", "moe_combine",
            "moe_load_stats_workspace_size", "moe_load_stats",
-           "moe_workspace_size", "moe_forward", "moe_forward_ex", "moe_forward_launches", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
+           "moe_workspace_size", "moe_forward", "moe_forward_ex", "moe_forward_launches",
+           "moe_set_fused_small_batch", "moe_check_status", "moe_debug_wait_timeout", "moe_num_sms", "moe_last_error")
 
 
 class MoeError(RuntimeError):
@@ -82,6 +83,7 @@ def load_library(path: str = LIB_PATH):
             "moe_forward_ex": (I, [P, I, P, P, P, F, I64, I, I, I, I, D, P, P, I, P, P, P, P, P, P, P, P, P, SZ,
                                    P]),
             "moe_forward_launches": (I, [I64, I, I, I, I, D, I]),
+            "moe_set_fused_small_batch": (I, [I]),
             "moe_check_status": (I, [P, P, ctypes.POINTER(U32)]),
             "moe_debug_wait_timeout": (I, [U32, P, SZ, P]),
             "moe_num_sms": (I, []),
@@ -380,6 +382,12 @@ def workspace_size(N, d, E, d_ff, k, cf, dtype) -> int:
 def forward_launches(N, d, E, d_ff, k, cf, dtype) -> int:
     dt = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32
     return int(load_library().moe_forward_launches(N, d, E, d_ff, k, _cf(cf), dt))
+
+
+def set_fused_small_batch(on: bool | None) -> bool:
+    """Select (True/False) or query (None) the single-launch small-batch layer
+    for this process; returns the previous setting."""
+    return bool(load_library().moe_set_fused_small_batch(-1 if on is None else int(bool(on))))
 
 
 def moe_forward(x, W_g, W_up, W_down, k, cf, b_g=None, noise=None, sigma=0.0, y=None, ws=None,

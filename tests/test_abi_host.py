@@ -4,6 +4,8 @@ import ctypes
 import math
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -132,3 +134,15 @@ def test_product_path_fails_loudly_without_the_library(tmp_path, monkeypatch):
     monkeypatch.setattr(moe, "_lib", None)
     with pytest.raises(ImportError):
         moe.load_library(str(tmp_path / "missing.so"))
+
+
+def test_fused_small_batch_off_by_default():
+    code = ("import sys; sys.path.insert(0, {root!r}); from sparse_mixture_experts_noisy_b200 import moe; "
+            "print(int(moe.set_fused_small_batch(None)))")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k != "MOE_FUSED_DECODE"}
+    r = subprocess.run([sys.executable, "-c", code.format(root=root)], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == "0"
+

@@ -1,7 +1,7 @@
 """The single-launch small-batch layer (decode_fused.cu) on the GPU (needs a B200).
 
-moe_forward runs batches of at most 64 bf16 tokens (E <= 16) as one
-cooperative kernel.  It must
+With moe_set_fused_small_batch(1), moe_forward runs batches of at most 64
+bf16 tokens (E <= 16) as one cooperative kernel.  It must
   - match the oracle (routing bit for bit on the GPU's logits, the output
     within the bf16 bar and the per-element rounding model),
   - give exactly the output of the separate kernels of the decode plan (the
@@ -54,6 +54,9 @@ np.save({out!r}, y.view(torch.int16).cpu().numpy())
 @pytest.fixture(scope="module", autouse=True)
 def _gpu():
     require_gpu()
+    prev = moe.set_fused_small_batch(True)
+    yield
+    moe.set_fused_small_batch(prev)
 
 
 def _kw(wl):
