@@ -1,9 +1,14 @@
 // Router building blocks shared by the router kernels (route_tc.cu) and the
 // fused small-batch layer (decode_fused.cu): the exact three-way bf16 split
 // of the fp32 router weights, the stage layout and MMAs of one K block, the
-// K pieces, the (hi + mid) + lo drain of a piece, and KeepTopK + softmax of
-// one token.  Both users run this same code, so a token's logits, picks and
-// gates come out bit for bit the same whichever kernel routed it.
+// K pieces, the drain of a piece, and KeepTopK + softmax of one token.  Both
+// users run this same code, so a token's logits, picks and gates come out bit
+// for bit the same whichever kernel routed it.
+//
+// Accumulators of one piece: 3 * E_pad fp32 columns of tensor memory, column
+// c summing the products with row c of B = [w_hi; w_mid; w_lo] (one MMA of
+// N = 3 * E_pad per 16-wide K step: each step reads the x tile from shared
+// memory once).  The piece's value is (hi-sum + mid-sum) + lo-sum.
 //
 // "Mixture of Experts (MoE) 12段階極小ビジュアル解剖シミュレーター" STEP 2 and 4-6;
 // "nanoMoEの深層解剖" slides 11-13.
@@ -69,7 +74,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
 }
 
 template <int UPT>
-__host__ __device__ constexpr int route_nb() {  // rows of B = accumulator columns
+__host__ __device__ constexpr int route_nb() {  // rows of B: [w_hi; w_mid; w_lo]
+    return 3 * 16 * UPT;
+}
+template <int UPT>
+__host__ __device__ constexpr int route_acc_cols() {  // accumulator columns of one piece
     return 3 * 16 * UPT;
 }
 
@@ -137,13 +146,22 @@ __device__ __forceinline__ void split_stage(uint8_t *stage_gen, int et) {
     }
 }
 
-template <int UPT>
-__host__ __device__ constexpr uint32_t route_tmem_cols() {  // clustered: one buffer
-    return route_nb<UPT>() <= 64 ? 64 : route_nb<UPT>() <= 128 ? 128 : route_nb<UPT>() <= 256 ? 256 : 512;
+__host__ __device__ constexpr uint32_t tmem_alloc_cols(int cols) {  // a power of two, at least 32
+    return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 template <int UPT>
-__host__ __device__ constexpr uint32_t routep_tmem_cols() {  // persistent: two buffers
-    return 2 * route_nb<UPT>() <= 128 ? 128 : 2 * route_nb<UPT>() <= 256 ? 256 : 512;
+__host__ __device__ constexpr uint32_t route_tmem_cols() {  // clustered: one buffer
+    return tmem_alloc_cols(route_acc_cols<UPT>());
+}
+// Persistent form: piece buffers in tensor memory (up to 4), so the MMAs run
+// ahead of the drains by up to that many pieces.
+template <int UPT>
+__host__ __device__ constexpr int routep_nbuf() {
+    return 512 / route_acc_cols<UPT>() < 4 ? 512 / route_acc_cols<UPT>() : 4;
+}
+template <int UPT>
+__host__ __device__ constexpr uint32_t routep_tmem_cols() {
+    return tmem_alloc_cols(routep_nbuf<UPT>() * route_acc_cols<UPT>());
 }
 
 // Which K blocks piece c of S sums: [c*kb/S, (c+1)*kb/S).
@@ -159,8 +177,8 @@ __host__ __device__ inline int route_k_splits(int d) {
     return s < 1 ? 1 : (s > 8 ? 8 : s);
 }
 
-// MMAs of one stage into accumulator d_tmem (N = 3 * E_pad, issued in chunks
-// of at most 256 columns); acc0 = 0 starts the sum.
+// MMAs of one stage into the piece accumulator at d_tmem (N = 3 * E_pad,
+// issued in chunks of at most 256 columns); acc0 = true starts the piece.
 template <int UPT>
 __device__ __forceinline__ void mma_stage(uint32_t st, uint32_t d_tmem, bool acc0) {
     constexpr int NB = route_nb<UPT>();
@@ -169,8 +187,7 @@ __device__ __forceinline__ void mma_stage(uint32_t st, uint32_t d_tmem, bool acc
     for (int kk = 0; kk < kRK / 16; ++kk) {
 #pragma unroll
         for (int n0 = 0; n0 < NB; n0 += 256) {
-            constexpr int kChunk = NB < 256 ? NB : 256;
-            const int nn = (NB - n0) < kChunk ? (NB - n0) : kChunk;
+            const int nn = (NB - n0) < 256 ? (NB - n0) : 256;
             const uint64_t bd = smem_desc_sw128(st + kXTileBytes + static_cast<uint32_t>(n0) * 128u);
             // +32 bytes along K inside the swizzled row = +2 in the address field
             umma_bf16(d_tmem + static_cast<uint32_t>(n0), ad + 2 * kk, bd + 2 * kk, idesc_bf16_f32(kRM, nn),
@@ -179,24 +196,31 @@ __device__ __forceinline__ void mma_stage(uint32_t st, uint32_t d_tmem, bool acc
     }
 }
 
-// Sum of one piece for this thread's token row: (hi + mid) + lo per expert,
-// from accumulator columns taddr (+E_pad, +2 E_pad); run = piece sum (first
-// piece) or run + piece sum.
+// The piece sums of experts [16 ch, 16 ch + 16) for this thread's token row:
+// (hi + mid) + lo, from the piece accumulator at taddr.
 template <int UPT>
-__device__ __forceinline__ void drain_piece(uint32_t taddr, bool first, float (&run)[16 * UPT]) {
-    constexpr int E_PAD = 16 * UPT;
+__device__ __forceinline__ void piece_chunk(uint32_t taddr, int ch, float (&p)[16]) {
+    constexpr int EP = 16 * UPT;
+    uint32_t h[16], m[16], l[16];
+    tmem_ld_32x32b_x16(taddr + ch * 16, h);
+    tmem_ld_32x32b_x16(taddr + EP + ch * 16, m);
+    tmem_ld_32x32b_x16(taddr + 2 * EP + ch * 16, l);
+    tmem_wait_ld();
 #pragma unroll
-    for (int ch = 0; ch < UPT; ++ch) {
-        uint32_t h[16], m[16], l[16];
-        tmem_ld_32x32b_x16(taddr + ch * 16, h);
-        tmem_ld_32x32b_x16(taddr + E_PAD + ch * 16, m);
-        tmem_ld_32x32b_x16(taddr + 2 * E_PAD + ch * 16, l);
-        tmem_wait_ld();
+    for (int i = 0; i < 16; ++i)
+        p[i] = __fadd_rn(__fadd_rn(__uint_as_float(h[i]), __uint_as_float(m[i])), __uint_as_float(l[i]));
+}
+
+// Sum of one piece for this thread's token row into run: the piece sum
+// (first piece) or run + piece sum, for the experts of chunks [ch0, ch0 + NCH).
+template <int UPT, int NCH = UPT>
+__device__ __forceinline__ void drain_piece(uint32_t taddr, bool first, float (&run)[16 * NCH], int ch0 = 0) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float p = __fadd_rn(__fadd_rn(__uint_as_float(h[i]), __uint_as_float(m[i])), __uint_as_float(l[i]));
-            run[ch * 16 + i] = first ? p : __fadd_rn(run[ch * 16 + i], p);
-        }
+    for (int ch = 0; ch < NCH; ++ch) {
+        float p[16];
+        piece_chunk<UPT>(taddr, ch0 + ch, p);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) run[ch * 16 + i] = first ? p[i] : __fadd_rn(run[ch * 16 + i], p[i]);
     }
 }
 
@@ -229,11 +253,13 @@ __device__ __forceinline__ void pick_row_smem(const float *sr, int E, int k, flo
 }
 
 // The same for scores held in registers (s[0..E), E <= E_PAD; s is consumed).
-// Each score becomes a 64-bit key whose order is the pick order: high word
-// the score mapped to an unsigned that orders like the float (-0 taken as +0,
-// so equal floats give equal words), low word ~e (lower index ranks first on
-// ties).  A round takes the largest key below the previous pick, as 8
-// independent running maxima folded at the end.
+// Each score becomes a 32-bit word whose unsigned order is the float order
+// (-0 taken as +0, so equal floats give equal words; every finite score maps
+// above 0).  A round takes, among the experts not picked yet, the largest
+// word and the lowest index among equal words: eight running (word, index)
+// pairs over e = i, i + 8, ... (a later e replaces the pair only when its
+// word is strictly larger), folded with ties going to the lower index.
+// Picked experts are bits of a mask.
 __device__ __forceinline__ uint32_t ordered_bits(float v) {
     const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -242,36 +268,123 @@ __device__ __forceinline__ float from_ordered_bits(uint32_t u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-template <int E_PAD>
-__device__ __forceinline__ void pick_row_regs(float (&s)[E_PAD], int E, int k, float *pv_s, int32_t *ti,
-                                              float *gt) {
-    uint32_t u[E_PAD];
-#pragma unroll
-    for (int e = 0; e < E_PAD; ++e) u[e] = ordered_bits(s[e]);
-    uint64_t prev = ~0ull;  // the first round takes the largest key
-    for (int j = 0; j < k; ++j) {
-        uint64_t part[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part[i] = 0;
-#pragma unroll
-        for (int e = 0; e < E_PAD; ++e) {
-            const uint64_t key = (static_cast<uint64_t>(u[e]) << 32) | static_cast<uint32_t>(~e);
-            const uint64_t cand = (e < E && key < prev) ? key : 0ull;
-            part[e & 7] = cand > part[e & 7] ? cand : part[e & 7];
-        }
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-            for (int i = 0; i < w; ++i) part[i] = part[i + w] > part[i] ? part[i + w] : part[i];
-        const uint64_t best = part[0];
-        ti[j] = static_cast<int32_t>(~static_cast<uint32_t>(best));
-        pv_s[j] = from_ordered_bits(static_cast<uint32_t>(best >> 32));
-        prev = best;
-    }
+// Softmax over the k kept scores in pick order (the first is the largest).
+__device__ __forceinline__ void softmax_kept(const float *pv_s, int k, float *gt) {
     const float mx = pv_s[0];
     float sum = 0.0f;
     for (int j = 0; j < k; ++j) sum = __fadd_rn(sum, expf(__fsub_rn(pv_s[j], mx)));
     for (int j = 0; j < k; ++j) gt[j] = __fdiv_rn(expf(__fsub_rn(pv_s[j], mx)), sum);
+}
+
+template <int E_PAD>
+__device__ __forceinline__ void pick_row_regs(float (&s)[E_PAD], int E, int k, float *pv_s, int32_t *ti,
+                                              float *gt) {
+    constexpr int W = (E_PAD + 31) / 32;
+    uint32_t u[E_PAD];
+#pragma unroll
+    for (int e = 0; e < E_PAD; ++e) u[e] = e < E ? ordered_bits(s[e]) : 0u;  // 0: never picked
+    uint32_t picked[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) picked[w] = 0u;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bu[8];
+        int be[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            bu[i] = 0u;
+            be[i] = E_PAD;
+        }
+#pragma unroll
+        for (int e = 0; e < E_PAD; ++e) {
+            const bool taken = (picked[e >> 5] >> (e & 31)) & 1u;
+            if (!taken && u[e] > bu[e & 7]) {
+                bu[e & 7] = u[e];
+                be[e & 7] = e;
+            }
+        }
+        uint32_t best = bu[0];
+        int arg = be[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            if (bu[i] > best || (bu[i] == best && be[i] < arg)) {
+                best = bu[i];
+                arg = be[i];
+            }
+        }
+        ti[j] = arg;
+        pv_s[j] = from_ordered_bits(best);
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+            if ((arg >> 5) == w) picked[w] |= 1u << (arg & 31);
+    }
+    softmax_kept(pv_s, k, gt);
+}
+
+// KeepTopK over one part of a token's experts, [e0, e0 + H) of which those
+// below E count: k rounds as above, writing each round's word and expert index
+// (word 0 once the part has no expert left).  The two parts' lists, each in
+// pick order, merge into the token's picks (merge_picks).
+template <int H>
+__device__ __forceinline__ void pick_part_regs(float (&s)[H], int e0, int E, int k, uint32_t *wo, int32_t *io) {
+    constexpr int W = (H + 31) / 32;
+    uint32_t u[H];
+#pragma unroll
+    for (int e = 0; e < H; ++e) u[e] = e0 + e < E ? ordered_bits(s[e]) : 0u;
+    uint32_t picked[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) picked[w] = 0u;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bu[8];
+        int be[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            bu[i] = 0u;
+            be[i] = H;
+        }
+#pragma unroll
+        for (int e = 0; e < H; ++e) {
+            const bool taken = (picked[e >> 5] >> (e & 31)) & 1u;
+            if (!taken && u[e] > bu[e & 7]) {
+                bu[e & 7] = u[e];
+                be[e & 7] = e;
+            }
+        }
+        uint32_t best = bu[0];
+        int arg = be[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            if (bu[i] > best || (bu[i] == best && be[i] < arg)) {
+                best = bu[i];
+                arg = be[i];
+            }
+        }
+        wo[j] = best;
+        io[j] = e0 + arg;
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+            if ((arg >> 5) == w) picked[w] |= 1u << (arg & 31);
+    }
+}
+
+// The token's k picks from the pick lists of its lower experts (a) and its
+// upper experts (b), each in pick order: a merge of the two orders, equal
+// words going to a (its experts have the lower indices).  Scores to pv_s,
+// experts to ti.
+__device__ __forceinline__ void merge_picks(const uint32_t *aw, const int32_t *ai, const uint32_t *bw,
+                                            const int32_t *bi, int k, float *pv_s, int32_t *ti) {
+    int i = 0, j = 0;
+    for (int n = 0; n < k; ++n) {
+        const uint32_t wa = i < k ? aw[i] : 0u, wb = j < k ? bw[j] : 0u;
+        if (wa >= wb) {
+            ti[n] = ai[i];
+            pv_s[n] = from_ordered_bits(wa);
+            ++i;
+        } else {
+            ti[n] = bi[j];
+            pv_s[n] = from_ordered_bits(wb);
+            ++j;
+        }
+    }
 }
 
 }  // namespace

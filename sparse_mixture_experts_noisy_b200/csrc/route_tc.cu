@@ -18,8 +18,8 @@
 // Tile: 128 tokens (MMA M) x all experts.  B is the 3*E_pad rows
 // [w_hi of experts 0..E_pad-1; w_mid ...; w_lo ...] of one 64-wide K block in
 // the 128-byte-swizzled K-major layout the MMA reads.  Accumulators: 3*E_pad
-// fp32 columns of tensor memory (column c = row c of B).  B comes one of two
-// ways:
+// fp32 columns of tensor memory per piece (column c = row c of B).  B comes
+// one of two ways:
 //   - pre-split: a first small kernel writes the parts of all of W_g, once per
 //     call, to a [3*E_pad, d] bf16 scratch, and TMA loads B beside the x tile
 //     (the fused forward, which has a workspace);
@@ -34,7 +34,7 @@
 //   - clustered (few tiles): the S CTAs of a cluster each sum one piece of one
 //     tile and exchange the sums through distributed shared memory;
 //   - persistent (many tiles): one CTA per SM walks whole tiles, each piece in
-//     its own tensor-memory buffer (two, so MMAs and drains overlap).
+//     one of up to four tensor-memory buffers, so MMAs and drains overlap.
 // Every wait is bounded; on expiry the kernel records ST_TIMEOUT, lets copies
 // and MMAs in flight land, writes expert -1 and gate 0 for its tokens, frees
 // its tensor memory and exits.
@@ -53,6 +53,7 @@ namespace {
 using namespace rt;
 
 constexpr int kRMaxStages = 8;
+constexpr int kRMaxBuf = 4;                        // persistent form: piece buffers
 constexpr int kRouteTcMaxE = 160;                  // 3 * E_pad <= 512 TMEM columns
 constexpr int kRouteTcMaxK = 32;                   // pick scratch: k floats per token
 constexpr size_t kRouteSmemBudget = 110 * 1024;    // per CTA: two CTAs fit on an SM
@@ -70,6 +71,7 @@ struct RouteTcArgs {
     int d, E, k, stages;
     int splits;    // S: pieces of K
     int pick_off;  // byte offset of the pick scratch: k floats per token row of a tile
+    int list_off;  // persistent form with two epilogue groups: byte offset of the pick lists
     float *logits_out;
     int32_t *topk_idx;
     float *gates;
@@ -130,7 +132,6 @@ template <int UPT, bool PRE>
 __global__ void __launch_bounds__(192, (PRE || UPT <= 2) ? 2 : 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                 const RouteTcArgs args) {
-    constexpr int E_PAD = 16 * UPT;
     constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
     constexpr uint32_t TMEM_COLS = route_tmem_cols<UPT>();
     static_assert(STAGE % 1024 == 0, "stage alignment");
@@ -287,17 +288,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll
             for (int ch = 0; ch < UPT; ++ch) {
-                uint32_t h[16], m[16], l[16];
-                tmem_ld_32x32b_x16(taddr + ch * 16, h);
-                tmem_ld_32x32b_x16(taddr + E_PAD + ch * 16, m);
-                tmem_ld_32x32b_x16(taddr + 2 * E_PAD + ch * 16, l);
-                tmem_wait_ld();
+                float p[16];
+                piece_chunk<UPT>(taddr, ch, p);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int e = ch * 16 + i;
-                    if (e < E)
-                        part[row * ld + e] = __fadd_rn(__fadd_rn(__uint_as_float(h[i]), __uint_as_float(m[i])),
-                                                       __uint_as_float(l[i]));
+                    if (e < E) part[row * ld + e] = p[i];
                 }
             }
         } else if (lane == 0) {
@@ -370,33 +366,50 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 // (at most 128, the MMA's M): the launcher picks it so that every CTA gets the
 // same number of tiles, and the MMA rows past tile_rows are computed on
 // whatever the stage holds there and never read.  A token's sums do not
-// depend on which rows share its tile.  Each piece of a tile sums from
-// zero into one of two tensor-memory buffers; the epilogue adds the piece sums
-// in order in registers, so each token gets what the clustered form gives it.
+// depend on which rows share its tile.  Piece p of the CTA (counting over its
+// tiles) sums from zero into tensor-memory buffer p % NBUF; the epilogue adds
+// the piece sums in order in registers, so each token gets what the clustered
+// form gives it.
 //
 // Warp roles: warp 0 lane 0 loads stages by TMA; warp 1 owns the tensor
-// memory and its lane 0 issues the MMAs; warps 2-5 drain the accumulators
-// (one token row per thread) and finish each tile (bias, logits, noise,
-// KeepTopK, softmax); warps 6-9 (in-kernel split only) split W_g into the B
-// slots.
-template <bool PRE>
+// memory and its lane 0 issues the MMAs; an epilogue group of four warps
+// drains the accumulators (one token row per thread) and finishes a tile
+// (bias, logits, noise, KeepTopK, softmax).  With pre-split weights and
+// E_pad <= 64, warps 2-5 and 6-9 are two epilogue groups taking alternate
+// tiles, so one group's finish overlaps the other's drains (320 threads,
+// which leaves a thread 168 registers: enough for 64 experts' sums and pick
+// words).  With the in-kernel split, warps 2-5 are the one group and warps
+// 6-9 split W_g into the B slots; E_pad = 80 with pre-split weights runs one
+// group in 192 threads.
+template <int UPT, bool PRE>
+__host__ __device__ constexpr int routep_groups() {
+    return (PRE && (UPT == 2 || UPT == 4)) ? 2 : 1;
+}
+
+// Barrier over the eight epilogue warps (id 2).
+__device__ __forceinline__ void epilogue_pair_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
+template <int UPT, bool PRE>
 __host__ __device__ constexpr int routep_threads() {
-    return PRE ? 192 : 320;
+    return 64 + 128 * routep_groups<UPT, PRE>() + (PRE ? 0 : 128);
 }
 
 template <int UPT, bool PRE>
-__global__ void __launch_bounds__(routep_threads<PRE>(), 1)
+__global__ void __launch_bounds__(routep_threads<UPT, PRE>(), 1)
 route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                  const RouteTcArgs args) {
-    constexpr int E_PAD = 16 * UPT;
-    constexpr int NB = route_nb<UPT>();
+    constexpr int ACC = route_acc_cols<UPT>();
+    constexpr int NBUF = routep_nbuf<UPT>();
+    constexpr int NG = routep_groups<UPT, PRE>();
+    constexpr int NCH = UPT / NG;  // 16-expert chunks one epilogue thread handles
+    constexpr int HE = 16 * NCH;
+    static_assert(NCH * NG == UPT, "the groups split the chunks evenly");
     constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
     constexpr uint32_t TMEM_COLS = routep_tmem_cols<UPT>();
-    static_assert(2 * NB <= 512, "two accumulator buffers");
+    static_assert(NBUF >= 2 && NBUF <= kRMaxBuf, "piece buffers");
     static_assert(STAGE % 1024 == 0, "stage alignment");
 
     extern __shared__ uint8_t dyn_smem[];
-    __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 5];
+    __shared__ __align__(8) uint64_t bars[3 * kRMaxStages + 2 * kRMaxBuf + 1];
     __shared__ uint32_t tmem_holder;
     __shared__ uint32_t cta_status;  // this CTA's copy of the status word
 
@@ -415,9 +428,9 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     const uint32_t xfull0 = smem_u32(&bars[0]);
     const uint32_t wfull0 = smem_u32(&bars[kRMaxStages]);
     const uint32_t empty0 = smem_u32(&bars[2 * kRMaxStages]);
-    const uint32_t accf0 = smem_u32(&bars[3 * kRMaxStages]);      // [2] piece sum ready
-    const uint32_t acce0 = smem_u32(&bars[3 * kRMaxStages + 2]);  // [2] buffer drained
-    const uint32_t drain = smem_u32(&bars[3 * kRMaxStages + 4]);
+    const uint32_t accf0 = smem_u32(&bars[3 * kRMaxStages]);             // [NBUF] piece sum ready
+    const uint32_t acce0 = smem_u32(&bars[3 * kRMaxStages + kRMaxBuf]);  // [NBUF] buffer drained
+    const uint32_t drain = smem_u32(&bars[3 * kRMaxStages + 2 * kRMaxBuf]);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -425,9 +438,9 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             mbar_init(wfull0 + 8 * s, 4);
             mbar_init(empty0 + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(accf0 + 8 * b, 1);
-            mbar_init(acce0 + 8 * b, 4);
+            mbar_init(acce0 + 8 * b, 4 * NG);  // every epilogue warp
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -492,15 +505,15 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             bool ok = true, any = false;
             for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
                 for (int c = 0; c < S && ok; ++c, ++piece) {
-                    const int b = piece & 1;
-                    const uint32_t use = static_cast<uint32_t>(piece >> 1);
+                    const int b = piece % NBUF;
+                    const uint32_t use = static_cast<uint32_t>(piece / NBUF);
                     if (!mbar_wait_bounded(acce0 + 8 * b, (use & 1u) ^ 1u, status, tmo, 22)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int kb0 = route_kb_begin(c, S, kb_total), kb1 = route_kb_begin(c + 1, S, kb_total);
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * NB);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * ACC);
                     for (int kb = kb0; kb < kb1; ++kb) {
                         if (!mbar_wait_bounded(xfull0 + 8 * stage, phase, status, tmo, 23) ||
                             (!PRE && !mbar_wait_bounded(wfull0 + 8 * stage, phase, status, tmo, 24))) {
@@ -524,7 +537,7 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 wait_until(drain, 0, tmo);
             }
         }
-    } else if (warp >= 6) {
+    } else if (!PRE && warp >= 6) {
         // ------------------------------------------------ W_g split into the B slots
         if constexpr (!PRE) {
             const int et = threadIdx.x - 192;  // 0..127
@@ -549,78 +562,139 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 2-5)
-        const int q = warp & 3;    // TMEM lane quarter
+        // ------------------------------------------------ epilogue group g (warps 2-5, 6-9)
+        // Group g drains and finishes the experts [g HE, (g + 1) HE) of every
+        // token of every tile (one token row per thread).
+        const int g = (warp - 2) >> 2;
+        const int q = warp & 3;  // TMEM lane quarter
         const int row = q * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-        float *pick_s = reinterpret_cast<float *>(smem_gen + args.pick_off);  // [128][k]
+        const int e0 = g * HE;
+        float *pv = reinterpret_cast<float *>(smem_gen + args.pick_off) + row * k;  // [128][k] kept scores
         const bool use_noise = (args.noise != nullptr) && (args.sigma != 0.0f);
-        int piece = 0;
+        const bool vec4 = (E & 3) == 0;  // rows of E floats are 16-byte aligned
         bool ok = true;
-        for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            float run[E_PAD];
+        int piece = 0, tt = 0;
+        for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tt) {
+            const int64_t t = tile * tile_rows + row;
+            const bool mine = row < tile_rows && t < args.N;
+            float run[HE];
+            float eps[NG == 2 ? HE : 1];  // this token's noise (its part), loaded while the last piece's MMAs run
             for (int c = 0; c < S; ++c, ++piece) {
-                const int b = piece & 1;
-                const uint32_t use = static_cast<uint32_t>(piece >> 1);
+                if constexpr (NG == 2) {
+                  if (c == S - 1 && use_noise && mine) {
+                    const float *nz = args.noise + t * E + e0;
+#pragma unroll
+                    for (int e = 0; e < HE; e += 4) {
+                        if (vec4) {
+                            if (e0 + e < E) {
+                                const float4 f = *reinterpret_cast<const float4 *>(nz + e);
+                                eps[e] = f.x; eps[e + 1] = f.y; eps[e + 2] = f.z; eps[e + 3] = f.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v)
+                                if (e0 + e + v < E) eps[e + v] = nz[e + v];
+                        }
+                    }
+                  }
+                }
+                const int b = piece % NBUF;
+                const uint32_t use = static_cast<uint32_t>(piece / NBUF);
                 ok = __all_sync(0xffffffffu, ok);
                 if (ok) ok = mbar_wait_warp(accf0 + 8 * b, use & 1u, status, tmo, 26);
                 tc_fence_after();
-                if (ok) drain_piece<UPT>(tmem_base + lane_off + static_cast<uint32_t>(b * NB), c == 0, run);
+                if (ok)
+                    drain_piece<UPT, NCH>(tmem_base + lane_off + static_cast<uint32_t>(b * ACC), c == 0, run, g * NCH);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acce0 + 8 * b);
             }
-            // finish this thread's token: bias, logits out, noise, KeepTopK, softmax
-            const int64_t t = tile * tile_rows + row;
-            if (row < tile_rows && t < args.N) {
-                int32_t *ti = args.topk_idx + t * k;
-                float *gt = args.gates + t * k;
-                if (ok) {
-                    if (args.b_g) {
+            // finish this thread's part of the token: bias, logits out, noise
+            if (mine && ok) {
+                if (args.b_g) {
 #pragma unroll
-                        for (int e = 0; e < E_PAD; ++e)
-                            if (e < E) run[e] = __fadd_rn(run[e], args.b_g[e]);
-                    }
-                    const bool vec4 = (E & 3) == 0;  // rows of E floats are 16-byte aligned
-                    if (args.logits_out) {
-                        float *lo = args.logits_out + t * E;
+                    for (int e = 0; e < HE; ++e)
+                        if (e0 + e < E) run[e] = __fadd_rn(run[e], args.b_g[e0 + e]);
+                }
+                if (args.logits_out) {
+                    float *lo = args.logits_out + t * E + e0;
 #pragma unroll
-                        for (int e = 0; e < E_PAD; e += 4) {
-                            if (vec4) {
-                                if (e < E)
-                                    *reinterpret_cast<float4 *>(lo + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
-                            } else {
+                    for (int e = 0; e < HE; e += 4) {
+                        if (vec4) {
+                            if (e0 + e < E)
+                                *reinterpret_cast<float4 *>(lo + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+                        } else {
 #pragma unroll
-                                for (int v = 0; v < 4; ++v)
-                                    if (e + v < E) lo[e + v] = run[e + v];
-                            }
+                            for (int v = 0; v < 4; ++v)
+                                if (e0 + e + v < E) lo[e + v] = run[e + v];
                         }
                     }
-                    if (use_noise) {
+                }
+                if (use_noise) {
+                    if constexpr (NG == 1) {
                         const float *nz = args.noise + t * E;
 #pragma unroll
-                        for (int e = 0; e < E_PAD; e += 4) {
-                            float q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        for (int e = 0; e < HE; e += 4) {
+                            float q4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                             if (vec4) {
                                 if (e < E) {
                                     const float4 f = *reinterpret_cast<const float4 *>(nz + e);
-                                    q[0] = f.x; q[1] = f.y; q[2] = f.z; q[3] = f.w;
+                                    q4[0] = f.x; q4[1] = f.y; q4[2] = f.z; q4[3] = f.w;
                                 }
                             } else {
 #pragma unroll
                                 for (int v = 0; v < 4; ++v)
-                                    if (e + v < E) q[v] = nz[e + v];
+                                    if (e + v < E) q4[v] = nz[e + v];
                             }
 #pragma unroll
                             for (int v = 0; v < 4; ++v)
-                                if (e + v < E) run[e + v] = __fadd_rn(run[e + v], __fmul_rn(args.sigma, q[v]));
+                                if (e + v < E) run[e + v] = __fadd_rn(run[e + v], __fmul_rn(args.sigma, q4[v]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < HE; ++e)
+                            if (e0 + e < E) run[e] = __fadd_rn(run[e], __fmul_rn(args.sigma, eps[e]));
+                    }
+                }
+            }
+            // KeepTopK and softmax
+            int32_t *ti = args.topk_idx + t * k;
+            float *gt = args.gates + t * k;
+            if constexpr (NG == 1) {
+                if (mine) {
+                    if (ok) {
+                        pick_row_regs<HE>(run, E, k, pv, ti, gt);
+                    } else {
+                        for (int j = 0; j < k; ++j) {
+                            ti[j] = -1;
+                            gt[j] = 0.0f;
                         }
                     }
-                    pick_row_regs<E_PAD>(run, E, k, pick_s + row * k, ti, gt);
-                } else {
-                    for (int j = 0; j < k; ++j) {
-                        ti[j] = -1;
-                        gt[j] = 0.0f;
+                }
+            } else {
+                // each part's picks in pick order: part 0 to list 0, part 1 to list
+                // 1 or 2 by tile parity (part 0 of the next tile cannot be merged
+                // before this barrier of the next tile, so list 1 / 2 is free by
+                // the time part 1 writes it again)
+                uint32_t *lw = reinterpret_cast<uint32_t *>(smem_gen + args.list_off);  // [3][128][k]
+                int32_t *li = reinterpret_cast<int32_t *>(lw + 3 * kRM * k);            // [3][128][k]
+                const int list = g == 0 ? 0 : 1 + (tt & 1);
+                if (mine && ok)
+                    pick_part_regs<HE>(run, e0, E, k, lw + (list * kRM + row) * k, li + (list * kRM + row) * k);
+                epilogue_pair_sync();
+                if (g == 0 && mine) {
+                    const int other = 1 + (tt & 1);
+                    const bool good = ok && (*reinterpret_cast<volatile uint32_t *>(status) & ST_ABORT) == 0u;
+                    if (good) {
+                        merge_picks(lw + row * k, li + row * k, lw + (other * kRM + row) * k,
+                                    li + (other * kRM + row) * k, k, pv, ti);
+                        softmax_kept(pv, k, gt);
+                    } else {
+                        for (int j = 0; j < k; ++j) {
+                            ti[j] = -1;
+                            gt[j] = 0.0f;
+                        }
                     }
                 }
             }
@@ -634,6 +708,13 @@ route_tcp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+}
+
+// The persistent form keeps a token's E_pad running sums and its pick words
+// in registers: E_pad <= 64 at 320 threads (168 registers a thread), and
+// E_pad = 80 with pre-split weights at 192 threads.
+__host__ __device__ constexpr bool route_persistent_ok(int upt, bool pre) {
+    return upt <= 4 || (upt == 5 && pre);
 }
 
 template <int UPT, bool PRE, int KIND>  // KIND: 0 clustered, 1 persistent
@@ -692,8 +773,12 @@ template <int UPT, bool PRE>
 cudaError_t launch_persistent_t(const CUtensorMap &tm, const CUtensorMap &tw, RouteTcArgs a, int64_t tiles,
                                 int sms, cudaStream_t s) {
     constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
+    // kept scores [128][k] floats, then (two groups) the pick lists: words
+    // and indices [3][128][k] each
     const size_t pick_bytes = static_cast<size_t>(kRM) * a.k * sizeof(float);
-    const size_t fixed = pick_bytes + 1024;
+    const size_t list_bytes =
+        routep_groups<UPT, PRE>() == 2 ? 2 * 3 * static_cast<size_t>(kRM) * a.k * sizeof(uint32_t) : 0;
+    const size_t fixed = pick_bytes + list_bytes + 1024;
     if (fixed + STAGE > kRpSmemBudget) return cudaErrorInvalidValue;
     int stages = static_cast<int>((kRpSmemBudget - fixed) / STAGE);
     if (stages > kRMaxStages) stages = kRMaxStages;
@@ -701,17 +786,18 @@ cudaError_t launch_persistent_t(const CUtensorMap &tm, const CUtensorMap &tw, Ro
     const size_t smem = ring + fixed;
     a.stages = stages;
     a.pick_off = static_cast<int>(ring);
+    a.list_off = static_cast<int>(ring + pick_bytes);
     auto kern = route_tcp_kernel<UPT, PRE>;
     cudaError_t e = set_smem_attr<UPT, PRE, 1>(kern, smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = tiles < sms ? tiles : sms;
-    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(routep_threads<PRE>()), smem, s, tm, tw, a);
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(routep_threads<UPT, PRE>()), smem, s, tm, tw, a);
 }
 
 template <int UPT, bool PRE>
 cudaError_t launch_form(bool persistent, const CUtensorMap &tm, const CUtensorMap &tw, const RouteTcArgs &a,
                         int64_t tiles, int sms, cudaStream_t s) {
-    if constexpr (2 * route_nb<UPT>() <= 512) {
+    if constexpr (route_persistent_ok(UPT, PRE) && routep_nbuf<UPT>() >= 2) {
         if (persistent) return launch_persistent_t<UPT, PRE>(tm, tw, a, tiles, sms, s);
     }
     return launch_cluster_t<UPT, PRE>(tm, tw, a, tiles, s);
@@ -773,16 +859,18 @@ cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, c
     CUtensorMap tm, tw;
     const int upt = route_upt(E);
     const int e_pad = 16 * upt, nb = 3 * e_pad;
-    RouteTcArgs a{b_g, noise, sigma, N, d, E, k, 0, route_k_splits(d), 0, logits_out, topk_idx, gates, status,
+    static_assert(routep_nbuf<5>() >= 2 && !route_persistent_ok(6, true), "persistent forms");
+    RouteTcArgs a{b_g, noise, sigma, N, d, E, k, 0, route_k_splits(d), 0, 0, logits_out, topk_idx, gates, status,
                   timeout_ns, kRM};
     int64_t tiles = (N + kRM - 1) / kRM;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // many tiles: the persistent form; few: clusters spread one tile's K over
     // up to 8 SMs
-    // (the persistent form needs two accumulator buffers of 3 * E_pad columns)
+    // (the persistent form holds up to 64, or 80 with pre-split weights,
+    // experts' sums in registers)
     const bool persistent = tiles * a.splits >= 2 * static_cast<int64_t>(sms) && route_tcp_enabled() &&
-                            2 * nb <= 512;
+                            route_persistent_ok(upt, w3 != nullptr);
     if (persistent) {
         // the same number of tiles on every SM: waves of full tiles, then the
         // tile height that spreads N evenly over that many waves
