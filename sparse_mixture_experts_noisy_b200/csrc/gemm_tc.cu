@@ -1008,6 +1008,283 @@ tc_wgrad_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant_
     }
 }
 
+// The weight gradients on CTA pairs (tcgen05 cta_group::2): a pair computes a
+// 256 x 256 tile of D[e], CTA r holding the M columns [r 128, r 128 + 128) of
+// the tile's P block (A) and the N columns [r 128, r 128 + 128) of its Q block
+// (B); the leader's MMA reads B from both CTAs and each CTA accumulates its 128
+// rows of D in its own tensor memory.  Per K block a CTA moves 32 KB through
+// TMA, where the one-CTA tile moves 48 KB for half the MMA work.
+// Both CTAs' loads complete on the leader's barrier (as in tc2_gemm_kernel).
+// The K rows past the expert's last row, in the last K block of a unit, are
+// zeroed by the leader's MMA warp in both CTAs' shared memory (the peer's
+// through the cluster window), behind a cluster-scope proxy fence, before it
+// issues that block's MMAs.
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+tc_wgrad2_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
+                 const WgArgs args) {
+    constexpr int BT = 256;                        // pair tile: 256 M x 256 N
+    constexpr uint32_t A_BYTES = 128 * kBK * 2;    // this CTA's 128 M columns: two 8 KB boxes
+    constexpr uint32_t B_BYTES = 128 * kBK * 2;    // this CTA's 128 N columns: two 8 KB boxes
+    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t TMEM_COLS = 512;            // two 256-column accumulators
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+    __shared__ uint32_t tmem_holder;
+    __shared__ int32_t cnt_s[256];
+    __shared__ int32_t off_s[256];
+    __shared__ uint32_t cta_status;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int E = args.E, M = args.M, Nn = args.Nn;
+    const int mt = (M + BT - 1) / BT, nt = (Nn + BT - 1) / BT;
+    const int total_units = E * mt * nt;
+    uint32_t *status = &cta_status;
+    const uint64_t tmo = args.timeout_ns;
+
+    const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    uint8_t *smem_gen = dyn_smem + (smem_base - smem_u32(dyn_smem));
+    const uint32_t full0 = smem_u32(&bars[0]);                // [STAGES] both CTAs' loads (leader's counts)
+    const uint32_t empty0 = smem_u32(&bars[STAGES]);          // [STAGES] the pair's MMAs are done
+    const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
+    const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+    const uint32_t full0_lead = map_to_cta(full0, 0);
+    const uint32_t tempty0_lead = map_to_cta(tempty0, 0);
+
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(tfull0, 1);
+        mbar_init(tfull0 + 8, 1);
+        mbar_init(tempty0, 8);  // 4 epilogue warps in each CTA
+        mbar_init(tempty0 + 8, 8);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+        cta_status = 0u;
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_p);
+        tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&tmem_holder), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        cnt_s[e] = args.counts[e];
+        off_s[e] = args.offsets[e];
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before either signals the other
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_holder;
+
+    auto decode = [&](int u, int &e, int &m, int &n) {
+        e = u / (mt * nt);
+        const int r = u - e * (mt * nt);
+        if (args.m_fast) {
+            m = r % mt;
+            n = r / mt;
+        } else {
+            m = r / nt;
+            n = r % nt;
+        }
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            const uint64_t pol = policy_evict_normal();
+            for (int u = pair; u < total_units && ok; u += npairs) {
+                int e, m, n;
+                decode(u, e, m, n);
+                const int nk = (cnt_s[e] + kBK - 1) / kBK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, status, tmo, 41)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * STAGE_BYTES);
+                    const uint32_t fb = full0_lead + 8 * stage;
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const int y = off_s[e] + kb * kBK;
+                    const int mc = m * BT + static_cast<int>(rank) * 128, nc = n * BT + static_cast<int>(rank) * 128;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) tma_load_2d_pair(sa + h * 8192u, &tm_p, fb, mc + h * 64, y, pol);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d_pair(sa + A_BYTES + h * 8192u, &tm_q, fb, nc + h * 64, y, pol);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {
+                // the pair's copies of the stages armed here land before exit
+                int st = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && i < issued; ++i) {
+                    if (st == 0) {
+                        st = STAGES - 1;
+                        ph ^= 1u;
+                    } else {
+                        --st;
+                    }
+                    wait_drain(full0 + 8 * st, ph, tmo);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ tail zeroing + MMA issue (leader, whole warp)
+        if (leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, any = false;
+            int local = 0;
+            const uint32_t idesc = idesc_bf16_f32(BT, BT) | kIdescAMajorMN | kIdescBMajorMN;
+            for (int u = pair; u < total_units && ok; u += npairs) {
+                int e, m, n;
+                decode(u, e, m, n);
+                const int cnt = cnt_s[e];
+                const int nk = (cnt + kBK - 1) / kBK;
+                if (nk == 0) continue;
+                const int acc = local & 1;
+                const uint32_t acc_phase = (local >> 1) & 1;
+                if (!mbar_wait_warp(tempty0 + 8 * acc, acc_phase ^ 1u, status, tmo, 42)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BT);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_warp(full0 + 8 * stage, phase, status, tmo, 43)) {
+                        ok = false;
+                        break;
+                    }
+                    const int v = cnt - kb * kBK;  // valid K rows of this block
+                    if (v < kBK) {
+                        // rows v.. of the four boxes, in this CTA and in the peer
+                        const uint32_t st = smem_base + stage * STAGE_BYTES;
+                        const uint32_t st_peer = map_to_cta(st, 1);
+                        const int per_box = (kBK - v) * 8;  // 16-byte chunks past the last row
+                        for (int q = lane; q < 4 * per_box; q += 32) {
+                            const int box = q / per_box, rem = q - box * per_box;
+                            const uint32_t off = static_cast<uint32_t>(box * 8192 + (v + rem / 8) * 128 + (rem % 8) * 16);
+                            *reinterpret_cast<uint4 *>(smem_gen + stage * STAGE_BYTES + off) = make_uint4(0u, 0u, 0u, 0u);
+                            st_shared_cluster_zero16(st_peer + off);
+                        }
+                        fence_proxy_async_smem();
+                        fence_proxy_async_cluster();  // the zeros, visible to the MMA in both CTAs
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                        const uint64_t ad = smem_desc_mn_sw128(sa, 8192u, 1024u);
+                        const uint64_t bd = smem_desc_mn_sw128(sa + A_BYTES, 8192u, 1024u);
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_bf16_pair(d_tmem, ad + 128u * kk, bd + 128u * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+                    }
+                    any = true;
+                    __syncwarp();
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) umma_commit_pair_mc(tfull0 + 8 * acc, 0x3);
+                ++local;
+            }
+            if (!ok && any && lane == 0) {
+                umma_commit_pair(drain);
+                wait_drain(drain, 0, tmo);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int u = pair; u < total_units; u += npairs) {
+            int e, m, n;
+            decode(u, e, m, n);
+            const int mrow = m * BT + static_cast<int>(rank) * 128 + row_in_tile;
+            float *o = args.out + (static_cast<int64_t>(e) * M + mrow) * Nn;
+            if (cnt_s[e] == 0) {
+                // no rows: a zero gradient, without touching the tensor memory
+                if (mrow < M)
+                    for (int c = n * BT; c < n * BT + BT && c < Nn; c += 4)
+                        *reinterpret_cast<float4 *>(o + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+                continue;
+            }
+            const int acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            if (!mbar_wait_warp(tfull0 + 8 * acc, acc_phase, status, tmo, 45)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BT);
+            for (int c = 0; c < BT / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_wait_ld();
+                const int col0 = n * BT + c * 32;
+                if (mrow < M) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int col = col0 + 4 * g;
+                        if (col < Nn)
+                            *reinterpret_cast<float4 *>(o + col) =
+                                make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                            __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(tempty0 + 8 * acc);
+                else mbar_arrive_cluster(tempty0_lead + 8 * acc);
+            }
+            ++local;
+        }
+    }
+    __syncwarp();
+    __syncthreads();
+    if (threadIdx.x == 0) publish_status(args.status, cta_status);
+    cluster_sync();  // the pair's MMAs and remote arrivals are done before the tensor memory goes
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+// MOE_WGRAD_PAIR=0 keeps the weight gradients on single CTAs (for comparisons).
+bool wgrad_pair_enabled() {
+    static const bool on = [] {
+        const char *v = getenv("MOE_WGRAD_PAIR");
+        return v == nullptr || atoi(v) != 0;
+    }();
+    return on;
+}
+
 cudaError_t launch_wgrad(const void *P, const void *Q, int64_t rows, int M, int Nn, const int32_t *offsets,
                          const int32_t *counts, int E, float *out, uint32_t *status, uint64_t timeout_ns,
                          int num_sms, cudaStream_t s) {
@@ -1019,9 +1296,20 @@ cudaError_t launch_wgrad(const void *P, const void *Q, int64_t rows, int M, int 
     auto kern = tc_wgrad_kernel<STAGES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    WgArgs a{offsets, counts, E, M, Nn, M <= Nn ? 1 : 0, out, status, timeout_ns};
+    if (num_sms >= 2 && wgrad_pair_enabled()) {
+        // CTA pairs, 256 x 256 tiles
+        constexpr int STAGES2 = 6;
+        constexpr int smem2 = STAGES2 * 2 * 128 * kBK * 2 + 1024;
+        auto kern2 = tc_wgrad2_kernel<STAGES2>;
+        e = cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+        if (e != cudaSuccess) return e;
+        const int units2 = E * ((M + 255) / 256) * ((Nn + 255) / 256);
+        const int pairs = units2 < num_sms / 2 ? units2 : num_sms / 2;
+        return launch_pdl(kern2, dim3(2 * (pairs > 0 ? pairs : 1)), dim3(kThreads), smem2, s, tm_p, tm_q, a);
+    }
     const int units = E * ((M + kWM - 1) / kWM) * ((Nn + kWN - 1) / kWN);
     const int grid = units < num_sms ? units : num_sms;
-    WgArgs a{offsets, counts, E, M, Nn, M <= Nn ? 1 : 0, out, status, timeout_ns};
     return launch_pdl(kern, dim3(grid > 0 ? grid : 1), dim3(kThreads), smem, s, tm_p, tm_q, a);
 }
 
