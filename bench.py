@@ -601,7 +601,10 @@ def run_ours(args):
             "e2e": {"value": wl.N * dist.world / e2e_sec, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": main["gpu_launches"],
-            "clocks": main["clocks"]}
+            "clocks": main["clocks"],
+            "router": main["router"]}
+    if main.get("single_launch"):
+        line["single_launch"] = main["single_launch"]
     del graphed
 
     if wl.dtype == "bf16" and not args.no_backward:

@@ -11,6 +11,9 @@ expert without rows must get exactly zero weight gradients.  The full-size
 case (the nanoMoE-shaped layer) is checked on sampled rows and columns that
 the oracle computes one by one, and on all of dW_g and db_g."""
 import math
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -181,3 +184,41 @@ def test_backward_full_size_nano():
     for key in ("dW_g", "db_g"):
         err = rel_err(g[key].cpu().numpy().astype(np.float64), ref[key])
         assert err <= tol, f"{key}: {err:.3g}"
+
+
+WGRAD_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r})
+from sparse_mixture_experts_noisy_b200.synth import WORKLOADS
+from tests.gpu_util import Case
+from tests.test_gpu_backward import CASES, make_dy, staged_train_step
+case = Case(CASES[{name!r}], seed=3)
+_, g = staged_train_step(case, make_dy(case.wl, 3))
+np.save({out_u!r}, g["dW_up"].cpu().numpy())
+np.save({out_d!r}, g["dW_down"].cpu().numpy())
+"""
+
+
+@pytest.mark.parametrize("name", ["ragged", "empty_experts", "fine_small"])
+def test_wgrad_one_cta_form_matches_pairs(name, tmp_path):
+    """The weight gradients on CTA pairs (the default) and on single CTAs
+    (MOE_WGRAD_PAIR=0, in a child process) agree to fp32 summation-order
+    rounding, expert by expert, and both give exact zeros to experts without
+    rows."""
+    case = Case(CASES[name], seed=3)
+    _, g = staged_train_step(case, make_dy(case.wl, 3))
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out_u, out_d = str(tmp_path / "u.npy"), str(tmp_path / "d.npy")
+    code = WGRAD_CHILD.format(root=root, name=name, out_u=out_u, out_d=out_d)
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=dict(os.environ, MOE_WGRAD_PAIR="0"),
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    for key, path in (("dW_up", out_u), ("dW_down", out_d)):
+        pair = g[key].cpu().numpy().astype(np.float64)
+        single = np.load(path).astype(np.float64)
+        for e in range(case.wl.E):
+            if not np.any(single[e]):
+                assert not np.any(pair[e]), f"{key}[{e}]"
+                continue
+            err = rel_err(pair[e], single[e])
+            assert err <= 1e-5, f"{key}[{e}]: {err:.3g}"
