@@ -310,17 +310,32 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         mbar_arrive_expect_tx(fb, kFWBytes);
                         tma_load_3d(smem_base + slot * kFSlot, phase == 0 ? &tm_wup : &tm_wdn, fb, kb * kRK, t.w0,
                                     t.e);
-                        const int q = ph % kFStages;
-                        pend_slot[q] = slot;
-                        pend_e[q] = t.e;
-                        pend_kb[q] = kb;
-                        pend_dn[q] = phase;
-                        ++ph;
+                        // once the phase's token rows exist and no earlier stage owes
+                        // its half, the token half goes with the weight half (the
+                        // queue below is only for the first stages of a phase)
+                        const bool both = pt == ph && (phase == 0 ? gathered : hready);
+                        if (both) {
+                            if (cnt_sm[t.e] > 0) {
+                                mbar_arrive_expect_tx(fb, kFTBytes);
+                                tma_load_2d(smem_base + slot * kFSlot + kFWBytes, phase == 0 ? &tm_xg : &tm_h, fb,
+                                            kb * kRK, off_sm[t.e]);
+                            } else {
+                                mbar_arrive(fb);  // no tokens: the MMA warp only releases the slot
+                            }
+                        } else {
+                            const int q = ph % kFStages;
+                            pend_slot[q] = slot;
+                            pend_e[q] = t.e;
+                            pend_kb[q] = kb;
+                            pend_dn[q] = phase;
+                            ++ph;
+                        }
                         gpar ^= 1u << slot;
                         if (++slot == kFStages) {
                             slot = 0;
                             ephase ^= 1u;
                         }
+                        if (both) continue;
                         // token halves that can go now without waiting
                         while (pt < ph && ((pend_dn[pt % kFStages] ? hready : gathered) ||
                                            ld_acquire_u32(a.sync + (pend_dn[pt % kFStages] ? SY_H : SY_GATHERED)) >=
@@ -595,15 +610,40 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 if (ok) {
                     const int64_t rows = a.offsets[E];
                     const int64_t total = rows * (d_ff / 4);
-                    for (int64_t i = static_cast<int64_t>(b) * 128 + et; i < total; i += static_cast<int64_t>(G) * 128) {
-                        float4 v = reinterpret_cast<const float4 *>(a.parts_up)[i];
-                        for (int p = 1; p < a.s_up; ++p) {
-                            const float4 w4 = reinterpret_cast<const float4 *>(a.parts_up + p * a.up_stride)[i];
-                            v.x += w4.x; v.y += w4.y; v.z += w4.z; v.w += w4.w;
+                    // eight 16-byte pieces per thread in flight at a time; each piece
+                    // sums the partials in split order
+                    constexpr int kB = 8;
+                    const int64_t step = static_cast<int64_t>(G) * 128;
+                    const float4 *pu = reinterpret_cast<const float4 *>(a.parts_up);
+                    for (int64_t i0 = static_cast<int64_t>(b) * 128 + et; i0 < total; i0 += kB * step) {
+                        float4 v[kB];
+#pragma unroll
+                        for (int j = 0; j < kB; ++j) {
+                            const int64_t i = i0 + j * step;
+                            v[j] = i < total ? pu[i] : make_float4(0.f, 0.f, 0.f, 0.f);
                         }
-                        __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(a.H) + 2 * i;
-                        o[0] = __floats2bfloat162_rn(fmaxf(v.x, 0.0f), fmaxf(v.y, 0.0f));
-                        o[1] = __floats2bfloat162_rn(fmaxf(v.z, 0.0f), fmaxf(v.w, 0.0f));
+                        for (int p = 1; p < a.s_up; ++p) {
+                            float4 w4[kB];
+                            const float4 *pp = reinterpret_cast<const float4 *>(a.parts_up + p * a.up_stride);
+#pragma unroll
+                            for (int j = 0; j < kB; ++j) {
+                                const int64_t i = i0 + j * step;
+                                w4[j] = i < total ? pp[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+#pragma unroll
+                            for (int j = 0; j < kB; ++j) {
+                                v[j].x += w4[j].x; v[j].y += w4[j].y; v[j].z += w4[j].z; v[j].w += w4[j].w;
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < kB; ++j) {
+                            const int64_t i = i0 + j * step;
+                            if (i < total) {
+                                __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(a.H) + 2 * i;
+                                o[0] = __floats2bfloat162_rn(fmaxf(v[j].x, 0.0f), fmaxf(v[j].y, 0.0f));
+                                o[1] = __floats2bfloat162_rn(fmaxf(v[j].z, 0.0f), fmaxf(v[j].w, 0.0f));
+                            }
+                        }
                     }
                 }
                 ok = epi_arrive(a, SY_H, et, &fail_s);
