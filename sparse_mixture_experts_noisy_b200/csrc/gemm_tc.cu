@@ -1379,8 +1379,10 @@ TcPlan plan_tc_ffn(int64_t rows, int d, int d_ff, int E, int num_sms) {
     if (p.decode) {
         // weight-streaming tiles: enough equal units that the last wave is a
         // small part of the whole, split over K (fp32 partials) to get there
-        // (the combine reads every down partial, so that one aims lower)
-        p.splits_up = decode_splits(static_cast<int64_t>(E) * ((d_ff + kBM - 1) / kBM), d, num_sms, 12);
+        // (the combine reads every down partial, so that one aims lower).  At
+        // the Mixtral shape the up projection's 896 weight tiles give 18.2
+        // waves with three splits, where two left 16 units in a 13th wave.
+        p.splits_up = decode_splits(static_cast<int64_t>(E) * ((d_ff + kBM - 1) / kBM), d, num_sms, 18);
         p.splits_down = decode_splits(static_cast<int64_t>(E) * ((d + kBM - 1) / kBM), d_ff, num_sms, 6);
     }
     return p;
