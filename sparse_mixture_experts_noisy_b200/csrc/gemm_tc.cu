@@ -49,7 +49,11 @@ constexpr int kThreads = 192;
 // bias and activation (up projection), raw fp32 partial sums (K splits; bias
 // and activation are applied once the splits are added), bf16 out zeroed
 // where a mask array is not positive (the ReLU's derivative in the backward).
-enum { EPI_BF16 = 0, EPI_BF16_ACT = 1, EPI_F32 = 2, EPI_BF16_MASK = 3 };
+// bf16 out (+ bias), bf16 out of bias + activation, fp32 partials, bf16 out
+// zeroed where a mask is not positive; and two fixed forms of the first two for
+// the layer without biases (ReLU only, nothing), whose epilogues carry no
+// runtime branches, and so much less code.
+enum { EPI_BF16 = 0, EPI_BF16_ACT = 1, EPI_F32 = 2, EPI_BF16_MASK = 3, EPI_BF16_RELU = 4, EPI_BF16_PLAIN = 5 };
 
 struct TcArgs {
     const int32_t *offsets;
@@ -75,7 +79,12 @@ __device__ __forceinline__ float activate(float v, int act) {
 // Weight-row tiles (swap = true): the lane's weight row w is fixed.
 template <int EPI, bool SWAP>
 __device__ __forceinline__ void bias_act(uint32_t (&r)[32], const TcArgs &args, int e, int col0, int w) {
-    if (EPI == EPI_F32) return;
+    if (EPI == EPI_F32 || EPI == EPI_BF16_PLAIN) return;
+    if (EPI == EPI_BF16_RELU) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
+        return;
+    }
     if (args.bias != nullptr) {
         const float *b = args.bias + static_cast<int64_t>(e) * args.Nw;
         if (SWAP) {
@@ -1412,9 +1421,16 @@ cudaError_t launch_tc_ffn(const void *xg, const int32_t *offsets, const int32_t 
     if (plan_out) *plan_out = p;
     cudaError_t e;
     if (!p.decode && p.pair) {
-        e = launch_tc2<EPI_BF16_ACT, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
-                                        timeout_ns, num_sms, s, b_up, act);
+        if (act == 1 && b_up == nullptr)
+            e = launch_tc2<EPI_BF16_RELU, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
+                                             timeout_ns, num_sms, s);
+        else
+            e = launch_tc2<EPI_BF16_ACT, 6>(xg, rows, W_up, E, d_ff, d, offsets, counts, H, d_ff, status,
+                                            timeout_ns, num_sms, s, b_up, act);
         if (e != cudaSuccess) return e;
+        if (b_down == nullptr)
+            return launch_tc2<EPI_BF16_PLAIN, 6>(H, rows, W_down, E, d, d_ff, offsets, counts, out, d, status,
+                                                 timeout_ns, num_sms, s);
         return launch_tc2<EPI_BF16, 6>(H, rows, W_down, E, d, d_ff, offsets, counts, out, d, status,
                                        timeout_ns, num_sms, s, b_down, 0);
     }
