@@ -79,7 +79,7 @@ __device__ __forceinline__ float activate(float v, int act) {
 // Weight-row tiles (swap = true): the lane's weight row w is fixed.
 template <int EPI, bool SWAP>
 __device__ __forceinline__ void bias_act(uint32_t (&r)[32], const TcArgs &args, int e, int col0, int w) {
-    if (EPI == EPI_F32 || EPI == EPI_BF16_PLAIN) return;
+    if (EPI == EPI_F32 || EPI == EPI_BF16_PLAIN || EPI == EPI_BF16_MASK) return;  // no bias, no activation
     if (EPI == EPI_BF16_RELU) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(fmaxf(__uint_as_float(r[i]), 0.0f));
@@ -1477,7 +1477,7 @@ cudaError_t launch_tc_bwd_gemms(const BwdArgs &a, const void *dO, void *dZ, void
                                                        dZ, a.d_ff, status, timeout_ns, num_sms, s, nullptr, 1, a.H);
     if (e != cudaSuccess) return e;
     // dX = dZ W_up[e]: tokens dZ [rows][d_ff] (K = d_ff), W_up [E][d_ff][d] read MN-major
-    e = launch_tc2<EPI_BF16, 6, true>(dZ, a.rows, a.W_up, a.E, a.d, a.d_ff, a.offsets, a.counts, dX, a.d, status,
+    e = launch_tc2<EPI_BF16_PLAIN, 6, true>(dZ, a.rows, a.W_up, a.E, a.d, a.d_ff, a.offsets, a.counts, dX, a.d, status,
                                       timeout_ns, num_sms, s);
     if (e != cudaSuccess) return e;
     // dW_down[e] = dO^T H ([d][d_ff]), dW_up[e] = dZ^T X ([d_ff][d])
