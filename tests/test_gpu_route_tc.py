@@ -159,6 +159,8 @@ PRESPLIT_CASES = {
     "e8_d4096": _wl("pe8", N=20000, d=4096, E=8, k=2, sigma=1.0, bias0=1.0),
     "e24_odd_tiles": _wl("pe24", N=30001, d=512, E=24, k=3, sigma=0.5, wg_std=0.1),
     "e64_fine": _wl("pe64", N=32768, d=2048, E=64, k=6, sigma=1.0),
+    # many picks per token: two groups' pick lists of 16 merged per token
+    "e64_k16": _wl("pe64k", N=20000, d=512, E=64, k=16, sigma=0.5, wg_std=0.05),
     "e80": _wl("pe80", N=40000, d=1024, E=80, k=4, sigma=0.5, wg_std=0.05, bias0=0.5),
 }
 
