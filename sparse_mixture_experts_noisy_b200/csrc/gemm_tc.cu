@@ -713,12 +713,9 @@ cudaError_t launch_tc(const void *tok, int64_t tok_rows, const void *W, int E, i
     if (!make_tmap_bf16_3d(&tm_w, W, E, Nw, K, SWAP ? kBM : BN)) return cudaErrorInvalidValue;
     constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024;
     auto kern = tc_gemm_kernel<BN, SWAP, EPI, STAGES>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // every call: the attribute belongs to the current device's context
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
     TcArgs a{offsets, counts, E, Nw, K, splits, out, ldo, split_stride, status, timeout_ns, bias, act, nullptr};
     return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, tm_tok, tm_w, a);
 }

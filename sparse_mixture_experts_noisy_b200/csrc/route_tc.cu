@@ -733,12 +733,15 @@ cudaError_t set_smem_attr(void (*kern)(CUtensorMap, CUtensorMap, RouteTcArgs), s
 }
 
 template <int UPT, bool PRE>
-cudaError_t launch_cluster_t(const CUtensorMap &tm, const CUtensorMap &tw, RouteTcArgs a, int64_t tiles,
+cudaError_t launch_cluster_t(const CUtensorMap &tm, const CUtensorMap &tw, RouteTcArgs a, int64_t tiles, int sms,
                              cudaStream_t s) {
     constexpr uint32_t STAGE = route_stage_bytes<UPT, PRE>();
-    // two CTAs per SM when two stages fit the half budget, else one CTA with
-    // as many stages as fit (one at least)
-    const size_t budget = (2 * STAGE + 1024 <= kRouteSmemBudget) ? kRouteSmemBudget : kRpSmemBudget;
+    // a grid that fits on the SMs at once: one CTA per SM with every stage it
+    // can hold (a piece's K blocks all in flight); else two CTAs per SM when
+    // two stages fit the half budget, else one CTA with as many stages as fit
+    const bool one_wave = tiles * a.splits <= sms;
+    const size_t budget =
+        (!one_wave && 2 * STAGE + 1024 <= kRouteSmemBudget) ? kRouteSmemBudget : kRpSmemBudget;
     int stages = static_cast<int>((budget - 1024) / STAGE);
     if (stages > kRMaxStages) stages = kRMaxStages;
     if (stages < 1) return cudaErrorInvalidValue;
@@ -750,7 +753,8 @@ cudaError_t launch_cluster_t(const CUtensorMap &tm, const CUtensorMap &tw, Route
     a.stages = stages;
     a.pick_off = static_cast<int>(part_bytes);
     auto kern = route_tc_kernel<UPT, PRE>;
-    cudaError_t e = set_smem_attr<UPT, PRE, 0>(kern, smem);
+    // the attribute is set once per device: to the largest request of any form
+    cudaError_t e = set_smem_attr<UPT, PRE, 0>(kern, kRpSmemBudget);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles * a.splits));
@@ -788,7 +792,7 @@ cudaError_t launch_persistent_t(const CUtensorMap &tm, const CUtensorMap &tw, Ro
     a.pick_off = static_cast<int>(ring);
     a.list_off = static_cast<int>(ring + pick_bytes);
     auto kern = route_tcp_kernel<UPT, PRE>;
-    cudaError_t e = set_smem_attr<UPT, PRE, 1>(kern, smem);
+    cudaError_t e = set_smem_attr<UPT, PRE, 1>(kern, kRpSmemBudget);  // once per device: the largest request
     if (e != cudaSuccess) return e;
     const int64_t grid = tiles < sms ? tiles : sms;
     return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(routep_threads<UPT, PRE>()), smem, s, tm, tw, a);
@@ -800,7 +804,7 @@ cudaError_t launch_form(bool persistent, const CUtensorMap &tm, const CUtensorMa
     if constexpr (route_persistent_ok(UPT, PRE) && routep_nbuf<UPT>() >= 2) {
         if (persistent) return launch_persistent_t<UPT, PRE>(tm, tw, a, tiles, sms, s);
     }
-    return launch_cluster_t<UPT, PRE>(tm, tw, a, tiles, s);
+    return launch_cluster_t<UPT, PRE>(tm, tw, a, tiles, sms, s);
 }
 
 template <bool PRE>

@@ -184,3 +184,19 @@ def test_router_pre_split_matches_in_kernel_split(name):
     assert torch.equal(t1, t2)
     assert torch.equal(g1.view(torch.int32), g2.view(torch.int32))
     _check(wl, inp, t1.cpu().numpy(), g1.cpu().numpy(), l1.cpu().numpy())
+
+
+def test_router_larger_k_after_smaller_in_one_process():
+    """The persistent router's shared memory grows with k (pick scratch and
+    pick lists); a call with a larger k after a smaller one must still launch
+    and route correctly (launch attributes are set once per device)."""
+    require_gpu()
+    for k in (2, 16, 4, 24):
+        wl = _wl(f"kgrow{k}", N=20000, d=256, E=64, k=k, sigma=0.5, wg_std=0.1)
+        inp = make_inputs(wl, seed=31 + k, weights=False)
+        x, W_g, b_g, noise = to_dev(inp.x), to_dev(inp.W_g), to_dev(inp.b_g), to_dev(inp.noise)
+        ws = moe.route_workspace(wl.d, wl.E, x.device)
+        t, g, lg = moe.moe_route(x, W_g, wl.k, b_g=b_g, noise=noise, sigma=wl.sigma, status=ws)
+        torch.cuda.synchronize()
+        assert moe.check_status(ws) == (0, 0)
+        _check(wl, inp, t.cpu().numpy(), g.cpu().numpy(), lg.cpu().numpy())
