@@ -375,12 +375,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 // memory and its lane 0 issues the MMAs; an epilogue group of four warps
 // drains the accumulators (one token row per thread) and finishes a tile
 // (bias, logits, noise, KeepTopK, softmax).  With pre-split weights and
-// E_pad <= 64, warps 2-5 and 6-9 are two epilogue groups taking alternate
-// tiles, so one group's finish overlaps the other's drains (320 threads,
-// which leaves a thread 168 registers: enough for 64 experts' sums and pick
-// words).  With the in-kernel split, warps 2-5 are the one group and warps
-// 6-9 split W_g into the B slots; E_pad = 80 with pre-split weights runs one
-// group in 192 threads.
+// E_pad = 32 or 64, warps 2-5 and 6-9 are two epilogue groups that both drain
+// every piece, group g for the experts [g E_pad/2, (g+1) E_pad/2): each picks
+// the top k of its half, and group 0 merges the two pick lists (320 threads,
+// 168 registers a thread).  With the in-kernel split, warps 2-5 are the one
+// group and warps 6-9 split W_g into the B slots; E_pad = 16 or 80 with
+// pre-split weights runs one group in 192 threads.
 template <int UPT, bool PRE>
 __host__ __device__ constexpr int routep_groups() {
     return (PRE && (UPT == 2 || UPT == 4)) ? 2 : 1;
