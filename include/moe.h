@@ -125,9 +125,10 @@ MOE_API size_t moe_route_workspace_size(int d, int E);
  *  - NULL: exactly moe_route (the library's status word);
  *  - ws_bytes >= 256: its first 4 bytes are the status word (zero before first
  *    use), read and cleared by moe_check_status(ws, ...);
- *  - ws_bytes >= moe_route_workspace_size(d, E), bf16 tokens: the router
- *    weights are also split into ws first and read from there (moe_forward's
- *    router: the persistent form on many tokens).  Same results either way. */
+ *  - ws_bytes >= moe_route_workspace_size(d, E), bf16 tokens: on batches that
+ *    take the router's persistent form (many tokens), the router weights are
+ *    also split into ws first and read from there, as in moe_forward; smaller
+ *    batches split them in-kernel.  Same results either way. */
 MOE_API moe_status moe_route_ex(const void *x, moe_dtype dt, const float *W_g, const float *b_g,
                                 const float *noise, float sigma, int64_t N, int d, int E, int k,
                                 float *logits_out, int32_t *topk_idx, float *gates, void *ws, size_t ws_bytes,

@@ -38,6 +38,9 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
                          cudaStream_t s, void *w3 = nullptr);
 // Kernels launch_route issues for 16-byte-aligned x and W_g (1, or 2 with w3
 // on the tensor-core path).
+// Whether a tensor-core router call with pre-split weights available reads
+// them (the persistent form) rather than splitting W_g in-kernel.
+bool route_tc_presplit_used(int64_t N, int d, int E, int sms);
 int route_launches(int dt, int64_t N, int d, int E, int k, bool with_w3);
 
 // Tensor-core router for bf16 tokens (route_tc.cu): same results contract as

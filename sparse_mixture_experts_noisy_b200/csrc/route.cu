@@ -392,7 +392,9 @@ cudaError_t launch_route(const void *x, int dt, const float *W_g, const float *b
 
 int route_launches(int dt, int64_t N, int d, int E, int k, bool with_w3) {
     if (N == 0) return 0;
-    return (dt == 1 && route_tc_shape_ok(N, d, E, k) && with_w3) ? 2 : 1;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return (dt == 1 && route_tc_shape_ok(N, d, E, k) && with_w3 && route_tc_presplit_used(N, d, E, sms)) ? 2 : 1;
 }
 
 }  // namespace moe

@@ -838,6 +838,15 @@ bool route_tcp_enabled() {
 
 }  // namespace
 
+// Whether a call with a pre-split workspace reads the split weights: only the
+// persistent form does.  The clustered form (few tiles) splits W_g in-kernel,
+// which gives the same bits and saves the split kernel's launch.
+bool route_tc_presplit_used(int64_t N, int d, int E, int sms) {
+    const int64_t tiles = (N + kRM - 1) / kRM;
+    return tiles * route_k_splits(d) >= 2 * static_cast<int64_t>(sms) && route_tcp_enabled() &&
+           route_persistent_ok(route_upt(E), true);
+}
+
 bool route_tc_shape_ok(int64_t N, int d, int E, int k) {
     static const bool enabled = [] {
         const char *v = getenv("MOE_ROUTE_TC");
@@ -869,6 +878,7 @@ cudaError_t launch_route_tc(const void *x, const float *W_g, const float *b_g, c
     int64_t tiles = (N + kRM - 1) / kRM;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (w3 != nullptr && !route_tc_presplit_used(N, d, E, sms)) w3 = nullptr;
     // many tiles: the persistent form; few: clusters spread one tile's K over
     // up to 8 SMs
     // (the persistent form holds up to 64, or 80 with pre-split weights,
