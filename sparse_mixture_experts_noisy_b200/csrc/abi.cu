@@ -35,13 +35,16 @@ moe_status cuda_fail(cudaError_t e, const char *where) {
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
 
 int num_sms_current() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];  // zero-initialised (static storage); any thread may fill an entry
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c != 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev < 64) cache[dev] = n;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
